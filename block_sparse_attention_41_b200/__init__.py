@@ -1,0 +1,6 @@
+"""Sol-Attn block-sparse attention forward for NVIDIA B200 (sm_100a).
+
+The compute path lives in the C-ABI shared library ``libsolattn.so`` (CUDA kernels under
+``csrc/``); :mod:`.sol_attn` is the thin ctypes binding with the same call names.
+:mod:`.workloads` draws the seeded synthetic inputs and does not touch the library.
+"""

@@ -1,0 +1,128 @@
+/*
+ * sol_attn.h -- C ABI of the Sol-Attn block-sparse attention forward for NVIDIA B200 (sm_100a).
+ *
+ * The operation: Sol-Attn project page ("Sol-Attn: Accelerating Video Generation Inference via
+ * On-the-Fly Attention Sparsification"), Abstract. One online-softmax pass does three things:
+ * it routes each query block to key blocks by a query-dependent threshold, selected on chip
+ * from a proxy score that is never written to memory; it runs exact attention on the kept
+ * blocks; and it adds an approximate correction for the skipped blocks. The Sol-Engine README,
+ * section "Sol-Attention", says the same: only the most relevant key blocks are computed, and
+ * a light compensating term covers the rest.
+ *
+ * Definition used (the pages give no formula; the CPU oracle follows the same one):
+ *   k_bar_j, v_bar_j = mean of K, V over the n_j valid tokens of key block j
+ *   q_bar_i          = mean of the valid query rows of query block i
+ *   s_bar_ij         = q_bar_i . k_bar_j / sqrt(d); keep j iff s_bar_ij >= max_j s_bar_ij - tau[h]
+ *                      or j < n_force
+ *   kept block       : exact logits q . k_t / sqrt(d), values v_t
+ *   skipped block    : one logit q . k_bar_j / sqrt(d) with multiplicity n_j, value v_bar_j
+ *   all terms of one query row share one softmax; attention is bidirectional (no causal mask).
+ *
+ * Conventions shared by every call:
+ *   - Tensors are dense, contiguous, row-major: [B, H, L, d] for Q, K, V, O (L = valid tokens, no
+ *     padding; partial last blocks are masked inside the kernels), [B, H, N_kb, d] for pooled
+ *     vectors, with N_kb = ceil(L / block_k) and N_qb = ceil(L / block_q).
+ *   - Device pointers must be 16-byte aligned. All device memory and the stream belong to the
+ *     caller; the library allocates nothing and keeps no global state.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). Every call
+ *     that launches work is asynchronous on that stream.
+ *   - Arguments are validated on the host before any launch. Invalid ones return SOL_EINVAL,
+ *     and shapes or dtypes the kernels do not implement return SOL_EUNSUPPORTED. In both cases
+ *     nothing is launched. A failed CUDA runtime call returns SOL_ECUDA.
+ *     sol_attn_last_error() gives the reason for the last failure on the calling thread.
+ *   - NaN or Inf inside Q, K, V is not checked and gives undefined results.
+ */
+#ifndef SOL_ATTN_H
+#define SOL_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SOL_OK = 0,
+    SOL_EINVAL = 1,        /* invalid argument (null pointer, bad size, tau < 0 or NaN, misalignment) */
+    SOL_EUNSUPPORTED = 2,  /* valid but not implemented (dtype / head dim / block size combination) */
+    SOL_ECUDA = 3,         /* a CUDA runtime call failed (launch, attribute, memset, copy) */
+    SOL_ETIMEOUT = 4       /* a bounded on-device wait expired; the kernel returned early (see check call) */
+} sol_status;
+
+typedef enum {
+    SOL_F32 = 0,  /* float32 inputs and output; SIMT kernel, fp32 arithmetic throughout */
+    SOL_BF16 = 1  /* bfloat16 inputs and output; tcgen05 tensor-core kernel, fp32 accumulation */
+} sol_dtype;
+
+/* Human-readable name of a status code. Never NULL. */
+const char* sol_attn_status_string(sol_status s);
+
+/* Detail of the most recent failing call on this thread ("" if none). Never NULL. */
+const char* sol_attn_last_error(void);
+
+/* Block pooling (definition of k_bar, v_bar above; Sol-Attn project page, Abstract: the routing
+ * proxy and the skipped-block correction both read pooled block vectors).
+ *
+ *   K, V      device, [B, H, L, d] in dtype `dt`
+ *   kbar,vbar device, float32 [B, H, N_kb, d]: mean over the n_j = min(block_k, L - j*block_k)
+ *             valid tokens of block j, summed in fp32
+ *   kbar_lp,  device, bfloat16 [B, H, N_kb, d]: the same means rounded to bf16 (nearest even),
+ *   vbar_lp   the operands of the tensor-core correction tiles. Required when dt == SOL_BF16,
+ *             must be NULL when dt == SOL_F32.
+ * Supported: SOL_BF16 with d % 8 == 0, SOL_F32 with d % 4 == 0, d <= 512, 1 <= block_k <= 4096.
+ */
+sol_status sol_attn_pool(const void* K, const void* V, sol_dtype dt, int B, int H, int L, int d,
+                         int block_k, float* kbar, float* vbar, void* kbar_lp, void* vbar_lp,
+                         void* stream);
+
+/* Bytes of device workspace sol_attn_fwd needs for this problem. The workspace holds the
+ * persistent scheduler's work counter, the per-(b,h) kept-block counters and the sticky
+ * device error word. Zero it once after allocation; later calls keep it consistent. */
+size_t sol_attn_fwd_workspace_bytes(int B, int H, int L, int block_q);
+
+/* The fused forward: routing, exact attention on kept blocks, skipped-block correction and the
+ * epilogue, in one kernel launch (Sol-Attn project page, Abstract).
+ *
+ *   Q, K, V     device, [B, H, L, d] in dtype `dt`
+ *   kbar        device, float32 [B, H, N_kb, d] from sol_attn_pool: the routing proxy
+ *   vbar        device, float32 [B, H, N_kb, d]: correction values for SOL_F32; may be NULL for
+ *               SOL_BF16
+ *   kbar_lp,    device, bf16 [B, H, N_kb, d] from sol_attn_pool: correction operands for
+ *   vbar_lp     SOL_BF16; ignored (may be NULL) for SOL_F32
+ *   tau         HOST, float32 [H]: per-head threshold, >= 0. +INFINITY keeps every block
+ *               (dense attention). Read during the call; the values travel in the launch.
+ *   block_q,    query / key block sizes. SOL_BF16: both 128, d in {64, 128}.
+ *   block_k     SOL_F32: equal, in {32, 64, 128}; d in {32, 64, 128}.
+ *   n_force     leading key blocks always kept (e.g. text tokens), 0 <= n_force <= N_kb
+ *   O           device, [B, H, L, d] in dtype `dt`: the output
+ *   kept_mask   device, uint8 [B, H, N_qb, N_kb] or NULL: 1 where block j was kept for query
+ *               block i
+ *   density     device, float32 [B, H] or NULL: kept blocks / (N_qb * N_kb) per head
+ *   workspace   device, >= sol_attn_fwd_workspace_bytes(...) bytes, zeroed once after allocation
+ * Limits: H <= 256, N_kb <= 4096, B*H*N_qb < 2^31.
+ * The proxy scores s_bar stay in shared memory and are never written to global memory.
+ */
+sol_status sol_attn_fwd(const void* Q, const void* K, const void* V, const float* kbar,
+                        const float* vbar, const void* kbar_lp, const void* vbar_lp,
+                        const float* tau, sol_dtype dt, int B, int H, int L, int d, int block_q,
+                        int block_k, int n_force, void* O, uint8_t* kept_mask, float* density,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then reads and clears the workspace's device error word. Returns
+ * SOL_ETIMEOUT if any launch since the last check gave up on a bounded wait, after which that
+ * launch's outputs are incomplete. Returns SOL_OK otherwise. */
+sol_status sol_attn_check_device_error(void* workspace, void* stream);
+
+/* Test hook for the failure-detection path. mode 0 (default) = normal operation. mode 1 makes
+ * the next sol_attn_fwd launch (SOL_BF16 path) skip one K-tile load, so the consumer's bounded
+ * wait expires: the launch returns early, sets the device error word, and
+ * sol_attn_check_device_error then reports SOL_ETIMEOUT. The hook applies to one launch and
+ * then resets to 0. The wait limit is about 0.2 s in that mode and about 2 s otherwise. */
+void sol_attn_debug_drop_one_load(int mode);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SOL_ATTN_H */

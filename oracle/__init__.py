@@ -1,0 +1,17 @@
+"""CPU oracle of the Sol-Attn forward. TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import
+this package. The CUDA library never calls it.
+"""
+from .sol_attn_oracle import (  # noqa: F401
+    BAND,
+    band_mask,
+    block_counts,
+    forward,
+    forward_head,
+    pool_blocks,
+    proxy_scores,
+    route,
+    unit_forward,
+    unit_terms,
+)
