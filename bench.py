@@ -1,0 +1,414 @@
+"""Benchmark of the Sol-Attn forward (block pooling + fused routing/exact/correction kernel).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--density D]
+
+One step = the whole hot path over one batch: sol_attn_pool (K/V block means) followed by
+sol_attn_fwd (routing, exact kept tiles, skipped-block correction, epilogue). It runs on the
+720p-like long-video workload (B=1, H=40, L=75,600, d=128, bf16, blocks of 128) at 20% kept
+blocks, with inputs resident in HBM. The metric is effective TFLOP/s over the kept tiles
+(4*128*128*d FLOPs per kept tile) per step, together with ms per step.
+
+Multi-GPU (torchrun): every rank runs an independent replica of the workload. There is no
+collective on the data path; per-rank times are reduced with MAX over ranks, and the value is
+the total work of all ranks divided by that time (weak scaling).
+
+`--impl reference` times the float64 CPU oracle on the host cores instead, on bounded samples
+of the same workload. That is the deliberately slow reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_attention_41_b200 import workloads as wl  # noqa: E402
+
+METRIC = "sparse-attn fwd ms & effective TFLOPS vs block density; % of bf16 tensor peak"
+DEFAULT_WORKLOAD = "video720p_L75600"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def tau_for(w, key):
+    with open(os.path.join(ROOT, "tests", "golden", "tau.json")) as f:
+        vals = json.load(f)["workloads"][w.name][key]["tau"]
+    return [math.inf if v == "inf" else float(v) for v in vals]
+
+
+def density_keys(w):
+    if w.per_head_density:
+        return ["per_head"]
+    return [str(x) for x in w.densities]
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {**FALLBACK_PEAKS, "bf16_tflops_sustained": FALLBACK_PEAKS["bf16_tflops"], "source": "fallback"}
+
+
+def kept_tile_flops(kept_blocks: int, w) -> float:
+    return 4.0 * w.block * w.block * w.d * kept_blocks
+
+
+# ------------------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu_id)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.path is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    mx = float(parts[1])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[4:8]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": []}
+        loaded = [s for s in sm if s >= 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------ CPU oracle
+def oracle_sample(w, tau, budget_s: float, max_units: int = 64, seed_offset: int = 77):
+    """Time the float64 oracle, as it stands, on seeded query-block units of the workload until
+    `budget_s` seconds of work are done. Returns (kept tiles processed, seconds, units, threads)."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # noqa: BLE001
+        threads = 1
+    units = wl.sample_units(w, max_units, seed_offset=seed_offset)
+    heads = {}
+    kept_tiles, elapsed, done = 0, 0.0, 0
+    for b, h, i in units:
+        if (b, h) not in heads:
+            heads = {(b, h): [x.astype(np.float64) for x in wl.head_tensors(w, b, h)]}
+        q, k, v = heads[(b, h)]
+        t0 = time.perf_counter()
+        _, keep, _, _ = oracle.forward_head(q, k, v, float(tau[h]), w.block, w.block, w.n_force, units=[i])
+        elapsed += time.perf_counter() - t0
+        kept_tiles += int(keep[i].sum())
+        done += 1
+        if elapsed >= budget_s:
+            break
+    return kept_tiles, elapsed, done, threads
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    key = args.density if args.density in density_keys(w) else density_keys(w)[0]
+    tau = tau_for(w, key)
+    per_step = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(w, tau, per_step * 0.25, seed_offset=1)
+    tiles, secs = 0, 0.0
+    units_done, threads = 0, 1
+    for s in range(args.steps):
+        t, e, u, threads = oracle_sample(w, tau, per_step, seed_offset=100 + s)
+        tiles += t
+        secs += e
+        units_done += u
+    tflops = kept_tile_flops(tiles, w) / secs / 1e12
+    line = {
+        "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "impl": "reference", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / max(args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d, "block": w.block,
+                   "density_target": key},
+        "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{units_done} seeded query-block units over {args.steps} steps "
+                                   f"(~{per_step:.0f} s of oracle work per step)"},
+        "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------------ GPU path
+def device_inputs(w, device, torch):
+    """Seeded inputs of the workload in HBM (heads drawn in a spawn-started process pool)."""
+    import multiprocessing as mp
+    from concurrent.futures import ProcessPoolExecutor
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    shape = (w.B, w.H, w.L, w.d)
+    Q, K, V = (torch.empty(shape, dtype=dt, device=device) for _ in range(3))
+    jobs = [(w.name, b, h) for b in range(w.B) for h in range(w.H)]
+    workers = max(1, min(len(jobs), (os.cpu_count() or 2) // max(1, int(os.environ.get("LOCAL_WORLD_SIZE", "1"))),
+                         32))
+    with ProcessPoolExecutor(max_workers=workers, mp_context=mp.get_context("spawn")) as ex:
+        for b, h, qkv in ex.map(wl._head_job, jobs):
+            for T, a in zip((Q, K, V), qkv):
+                T[b, h].copy_(torch.from_numpy(a).to(dt))
+    return Q, K, V
+
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+    from block_sparse_attention_41_b200 import sol_attn as sa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    sa.load_library()
+    Q, K, V = device_inputs(w, dev, torch)
+    keys = density_keys(w)
+    key = args.density if args.density in keys else ("0.2" if "0.2" in keys else keys[0])
+    tau = tau_for(w, key)
+    B, H, L, d, blk = w.B, w.H, w.L, w.d, w.block
+    nb = w.n_blocks
+    stream = torch.cuda.current_stream()
+    ws = sa.new_workspace(B, H, L, blk, dev)
+    kbar = torch.empty((B, H, nb, d), dtype=torch.float32, device=dev)
+    vbar = torch.empty_like(kbar)
+    klp = torch.empty((B, H, nb, d), dtype=torch.bfloat16, device=dev)
+    vlp = torch.empty_like(klp)
+    O = torch.empty_like(Q)
+    dens = torch.empty((B, H), dtype=torch.float32, device=dev)
+
+    def step(tau_v, ev=None):
+        sa.sol_attn_pool(K, V, blk, kbar, vbar, klp, vlp, stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        sa.sol_attn_fwd(Q, K, V, kbar, vbar, klp, vlp, tau_v, blk, blk, w.n_force, O=O, density=dens,
+                        workspace=ws, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    # kept blocks at the timed density (from the kernel's own density output)
+    step(tau)
+    torch.cuda.synchronize()
+    sa.sol_attn_check_device_error(ws)
+    kept = int(round(float(dens.double().sum()) * nb * nb))
+    flops = kept_tile_flops(kept, w)
+
+    for _ in range(args.warmup):
+        step(tau)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    fwd_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_gpu_index(torch, local)) as clk:
+        t0.record(stream)
+        for s in range(args.steps):
+            step(tau, fwd_ev[s])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    sa.sol_attn_check_device_error(ws)
+    ms_total = max_over_ranks(t0.elapsed_time(t1))
+    ms_step = ms_total / args.steps
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_ev)
+    value = world * flops / (ms_step * 1e-3) / 1e12
+    pk = peaks()
+    achieved = flops / (fwd_ms * 1e-3) / 1e12
+
+    # density sweep incl. dense (tau = +inf), untimed by the contract but measured the same way
+    sweep = []
+    if not args.no_sweep:
+        for kk in keys:
+            tv = tau_for(w, kk)
+            step(tv)
+            torch.cuda.synchronize()
+            kb = int(round(float(dens.double().sum()) * nb * nb))
+            n_it = 3
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_it)]
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for i in range(n_it):
+                step(tv, evs[i])
+            a1.record(stream)
+            torch.cuda.synchronize()
+            f_ms = statistics.mean(x.elapsed_time(y) for x, y in evs)
+            sweep.append({"density_target": kk, "density": kb / float(B * H * nb * nb),
+                          "ms_per_step": a0.elapsed_time(a1) / n_it, "fwd_ms": f_ms,
+                          "fwd_tflops": kept_tile_flops(kb, w) / (f_ms * 1e-3) / 1e12})
+        dense = [s for s in sweep if s["density_target"] == "1.0"]
+        if dense:
+            for s in sweep:
+                s["speedup_vs_dense"] = dense[0]["ms_per_step"] / s["ms_per_step"]
+
+    # end to end through the public API: pinned host inputs in, host output back, every step
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (Q, K, V))
+        ho = torch.empty_like(hq).pin_memory()
+        e_steps = max(1, min(args.steps, 5))
+
+        def e2e_step():
+            q = hq.to(dev, non_blocking=True)
+            k = hk.to(dev, non_blocking=True)
+            v = hv.to(dev, non_blocking=True)
+            o, _, _ = sa.sol_attn(q, k, v, tau, block=blk, n_force=w.n_force, workspace=ws, stream=stream)
+            ho.copy_(o, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = max_over_ranks(e0.elapsed_time(e1)) / e_steps
+        nbytes = Q.numel() * Q.element_size()
+        e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e_ms,
+               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes}
+        del hq, hk, hv, ho
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tiles, secs, units, threads = oracle_sample(w, tau, args.cpu_budget)
+        cpu = {"value": kept_tile_flops(tiles, w) / secs / 1e12, "unit": "TFLOP/s", "cores": threads,
+               "kind": "oracle",
+               "sample": f"{units} seeded query-block units of {w.name} at density {key} "
+                         f"({secs:.1f} s of float64 oracle work, extrapolated per kept tile)"}
+
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(prof):
+        with open(prof) as f:
+            tr = json.load(f)
+        if tr.get("workload") == w.name and tr.get("density") == key:
+            traffic = tr.get("bytes_per_launch")
+
+    if rank == 0:
+        clocks = clk.summary()
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": w.name, "B": B, "H": H, "L": L, "d": d, "block": blk,
+                       "density_target": key, "density": kept / float(B * H * nb * nb),
+                       "kept_tiles": kept, "n_force": w.n_force,
+                       "l2": "inputs (Q,K,V %.2f GB) larger than the 126 MB L2; no flush" %
+                             (3 * Q.numel() * Q.element_size() / 1e9),
+                       "parallelism": f"replica x{world}"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / pk["bf16_tflops"], "traffic": traffic,
+                         "kernel": "sol_fwd_tc_kernel", "fwd_ms": fwd_ms,
+                         "peak_source": f"{pk['source']} bf16 dense (burst)"},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 2 * args.steps,
+            "clocks": clocks,
+            "sweep": sweep,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def local_gpu_index(torch, local):
+    """nvidia-smi id of this process's GPU (its UUID, robust to CUDA_VISIBLE_DEVICES)."""
+    try:
+        u = str(torch.cuda.get_device_properties(local).uuid)
+        return u if u.startswith("GPU-") else f"GPU-{u}"
+    except Exception:  # noqa: BLE001
+        return local
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--density", default="0.2")
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = wl.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

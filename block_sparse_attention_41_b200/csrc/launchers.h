@@ -1,0 +1,42 @@
+// Internal launcher interface between the C ABI (sol_attn_api.cu) and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace sol {
+
+struct FwdArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  const float* kbar;
+  const float* vbar;
+  const void* kbar_lp;
+  const void* vbar_lp;
+  const float* tau;  // host [H]
+  bool bf16;
+  int B, H, L, d, block;
+  int n_force;
+  void* O;
+  uint8_t* kept_mask;
+  float* density;
+  uint32_t* ws;
+  int num_sms;
+  int drop_one_load;       // failure-detection test hook (bf16 path)
+  uint64_t wait_limit_ns;  // bound on every on-device wait
+};
+
+cudaError_t launch_pool(const void* K, const void* V, bool bf16, int BH, int L, int d, int block,
+                        float* kbar, float* vbar, void* kbar_lp, void* vbar_lp, cudaStream_t stream);
+
+// bf16, d in {64, 128}, block 128: TMA + tcgen05 persistent kernel.
+cudaError_t launch_fwd_tc(const FwdArgs& a, const CUtensorMap* maps /* Q, K, V, Kbar_lp, Vbar_lp */,
+                          cudaStream_t stream);
+
+// fp32, d in {32, 64, 128}, block in {32, 64, 128}: SIMT kernel.
+cudaError_t launch_fwd_simt(const FwdArgs& a, cudaStream_t stream);
+
+}  // namespace sol

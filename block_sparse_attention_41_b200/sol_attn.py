@@ -1,0 +1,208 @@
+"""Thin ctypes binding of libsolattn.so (C ABI in include/sol_attn.h), with the same call names.
+
+This module only marshals arguments: it checks tensor placement, dtype and contiguity,
+allocates output tensors with torch when the caller passes none, passes raw pointers and
+the current CUDA stream, and turns status codes into exceptions. All compute runs in the
+library's CUDA kernels. There is no fallback: if the library is missing or no sm_100 GPU is
+present, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Sequence
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsolattn.so")
+
+SOL_OK, SOL_EINVAL, SOL_EUNSUPPORTED, SOL_ECUDA, SOL_ETIMEOUT = range(5)
+SOL_F32, SOL_BF16 = 0, 1
+
+# symbols declared in include/sol_attn.h
+EXPORTED = (
+    "sol_attn_status_string",
+    "sol_attn_last_error",
+    "sol_attn_pool",
+    "sol_attn_fwd_workspace_bytes",
+    "sol_attn_fwd",
+    "sol_attn_check_device_error",
+    "sol_attn_debug_drop_one_load",
+)
+
+
+class SolAttnError(RuntimeError):
+    """A library call returned a status other than SOL_OK."""
+
+    def __init__(self, status: int, call: str, detail: str):
+        self.status = status
+        super().__init__(f"{call}: {status_string(status)}: {detail}")
+
+
+_lib = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libsolattn.so once; raise if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with `python -m block_sparse_attention_41_b200.build` "
+            "(there is no non-CUDA implementation)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, f32p = ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(ctypes.c_float)
+    lib.sol_attn_status_string.argtypes = [i32]
+    lib.sol_attn_status_string.restype = ctypes.c_char_p
+    lib.sol_attn_last_error.argtypes = []
+    lib.sol_attn_last_error.restype = ctypes.c_char_p
+    lib.sol_attn_pool.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp]
+    lib.sol_attn_pool.restype = i32
+    lib.sol_attn_fwd_workspace_bytes.argtypes = [i32, i32, i32, i32]
+    lib.sol_attn_fwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.sol_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, f32p, i32, i32, i32, i32, i32, i32, i32, i32,
+                                 vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.sol_attn_fwd.restype = i32
+    lib.sol_attn_check_device_error.argtypes = [vp, vp]
+    lib.sol_attn_check_device_error.restype = i32
+    lib.sol_attn_debug_drop_one_load.argtypes = [i32]
+    lib.sol_attn_debug_drop_one_load.restype = None
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().sol_attn_status_string(int(status)).decode()
+
+
+def _check(status: int, call: str) -> None:
+    if status != SOL_OK:
+        raise SolAttnError(status, call, load_library().sol_attn_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SOL_BF16
+    if t.dtype == torch.float32:
+        return SOL_F32
+    raise TypeError(f"unsupported dtype {t.dtype}: use torch.bfloat16 or torch.float32")
+
+
+def _need_cuda(name: str, t: torch.Tensor, dtype=None) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must have dtype {dtype}, got {t.dtype}")
+
+
+def sol_attn_pool(K: torch.Tensor, V: torch.Tensor, block_k: int, kbar=None, vbar=None, kbar_lp=None,
+                  vbar_lp=None, stream=None):
+    """Block means of K and V. Returns (kbar, vbar, kbar_lp, vbar_lp); the bf16 mirrors are None
+    for fp32 inputs."""
+    _need_cuda("K", K)
+    _need_cuda("V", V, K.dtype)
+    B, H, L, d = K.shape
+    if V.shape != K.shape:
+        raise ValueError("K and V must have the same shape")
+    nkb = -(-L // block_k)
+    dt = _dtype_code(K)
+    dev = K.device
+    if kbar is None:
+        kbar = torch.empty((B, H, nkb, d), dtype=torch.float32, device=dev)
+    if vbar is None:
+        vbar = torch.empty((B, H, nkb, d), dtype=torch.float32, device=dev)
+    if dt == SOL_BF16:
+        if kbar_lp is None:
+            kbar_lp = torch.empty((B, H, nkb, d), dtype=torch.bfloat16, device=dev)
+        if vbar_lp is None:
+            vbar_lp = torch.empty((B, H, nkb, d), dtype=torch.bfloat16, device=dev)
+    for n, t in (("kbar", kbar), ("vbar", vbar)):
+        _need_cuda(n, t, torch.float32)
+    st = load_library().sol_attn_pool(_ptr(K), _ptr(V), dt, B, H, L, d, block_k, _ptr(kbar), _ptr(vbar),
+                                      _ptr(kbar_lp), _ptr(vbar_lp), _stream(stream))
+    _check(st, "sol_attn_pool")
+    return kbar, vbar, kbar_lp, vbar_lp
+
+
+def sol_attn_fwd_workspace_bytes(B: int, H: int, L: int, block_q: int) -> int:
+    return int(load_library().sol_attn_fwd_workspace_bytes(B, H, L, block_q))
+
+
+def new_workspace(B: int, H: int, L: int, block_q: int, device) -> torch.Tensor:
+    """A zeroed workspace buffer of the size sol_attn_fwd needs."""
+    return torch.zeros(sol_attn_fwd_workspace_bytes(B, H, L, block_q), dtype=torch.uint8, device=device)
+
+
+def sol_attn_fwd(Q, K, V, kbar, vbar, kbar_lp, vbar_lp, tau: Sequence[float], block_q: int, block_k: int,
+                 n_force: int = 0, O=None, kept_mask=None, density=None, workspace=None, stream=None):
+    """Fused routing + exact kept-block attention + skipped-block correction. Returns O.
+
+    `tau` is a host sequence of H floats (>= 0, +inf = dense). `kept_mask` (uint8
+    [B,H,N_qb,N_kb]) and `density` (float32 [B,H]) are optional output tensors.
+    """
+    _need_cuda("Q", Q)
+    for n, t in (("K", K), ("V", V)):
+        _need_cuda(n, t, Q.dtype)
+    B, H, L, d = Q.shape
+    if K.shape != Q.shape or V.shape != Q.shape:
+        raise ValueError("Q, K and V must have the same shape [B, H, L, d]")
+    dt = _dtype_code(Q)
+    tau = [float(x) for x in tau]
+    if len(tau) != H:
+        raise ValueError(f"tau must hold H={H} values")
+    if O is None:
+        O = torch.empty_like(Q)
+    if workspace is None:
+        workspace = new_workspace(B, H, L, block_q, Q.device)
+    tau_c = (ctypes.c_float * H)(*tau)
+    st = load_library().sol_attn_fwd(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(kbar), _ptr(vbar), _ptr(kbar_lp), _ptr(vbar_lp), tau_c, dt, B, H, L, d,
+        block_q, block_k, int(n_force), _ptr(O), _ptr(kept_mask), _ptr(density), _ptr(workspace),
+        workspace.numel(), _stream(stream))
+    _check(st, "sol_attn_fwd")
+    return O
+
+
+def sol_attn_check_device_error(workspace: torch.Tensor, stream=None) -> None:
+    """Synchronise and raise SolAttnError(SOL_ETIMEOUT) if a bounded device wait expired."""
+    _check(load_library().sol_attn_check_device_error(_ptr(workspace), _stream(stream)),
+           "sol_attn_check_device_error")
+
+
+def sol_attn_debug_drop_one_load(mode: int) -> None:
+    load_library().sol_attn_debug_drop_one_load(int(mode))
+
+
+def sol_attn(Q, K, V, tau, block: int = 128, n_force: int = 0, want_mask: bool = False,
+             want_density: bool = False, workspace=None, stream=None):
+    """The whole path for one call: pool K/V, then the fused forward.
+
+    Returns (O, kept_mask or None, density or None).
+    """
+    B, H, L, d = Q.shape
+    kbar, vbar, kbar_lp, vbar_lp = sol_attn_pool(K, V, block, stream=stream)
+    nb = -(-L // block)
+    mask = torch.empty((B, H, nb, nb), dtype=torch.uint8, device=Q.device) if want_mask else None
+    dens = torch.empty((B, H), dtype=torch.float32, device=Q.device) if want_density else None
+    O = sol_attn_fwd(Q, K, V, kbar, vbar, kbar_lp, vbar_lp, tau, block, block, n_force, kept_mask=mask,
+                     density=dens, workspace=workspace, stream=stream)
+    return O, mask, dens
+
+
+def tau_list(values) -> list:
+    """Turn a JSON-style tau list ("inf" strings allowed) into floats."""
+    return [math.inf if (isinstance(v, str) and v.lower() == "inf") else float(v) for v in values]
