@@ -43,7 +43,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 def tau_for(w, key):
     with open(os.path.join(ROOT, "tests", "golden", "tau.json")) as f:
         vals = json.load(f)["workloads"][w.name][key]["tau"]
-    return [math.inf if v == "inf" else float(v) for v in vals]
+    return [math.inf if v == "inf" else float(v) for v in vals][: w.H]
 
 
 def density_keys(w):
@@ -401,10 +401,15 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--heads", type=int, default=0,
+                    help="profiling only: keep the first N heads of the workload (same seeds)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     w = wl.WORKLOADS[args.workload]
+    if args.heads:
+        import dataclasses
+        w = dataclasses.replace(w, H=min(args.heads, w.H))
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

@@ -14,18 +14,28 @@
 //                 MMA/softmax pipeline and the same running max, sum and accumulator.
 //   4. epilogue : O / l -> bf16 -> global.
 //
-// Roles (256 threads): warp 0 = TMA producer, warp 1 = MMA issuer (also owns TMEM),
-// warps 4..7 = router + softmax + epilogue (thread r owns query row r = TMEM lane r), warps 2..3
-// idle. Units come from an atomic counter in head-major order, so CTAs running at the same
-// time share one head's K/V in L2.
+// Roles (320 threads): warp 0 = TMA producer, warp 1 = MMA issuer (also owns TMEM), warps 2..5
+// and 6..9 = two softmax groups. A warp may only touch TMEM lanes 32*(warp%4) .. +31, and any four
+// consecutive warps cover all four quarters, so thread (g, r) of softmax group g owns query
+// row r (TMEM lane r) and score columns [64g, 64g+64). The two halves exchange their row max
+// once per tile through shared memory. Both groups also do the routing and the epilogue. Units
+// come from an atomic counter in head-major order, so CTAs running at the same time share one
+// head's K/V in L2.
 //
 // TMEM columns: S0 [0,128) S1 [128,256) O [256,256+D) P0 [384,448) P1 [448,512).
-// P has its own columns, separate from S. The next QK^T into S[b] therefore never has to wait
-// for the PV MMA that reads P[b].
+// P has its own columns, separate from S, so the QK^T that refills S[b] never races the PV MMA
+// that reads P[b]. K tiles go round a 3-deep ring (d = 128) and are released as soon as their
+// QK^T completes. V tiles go round a 2-deep ring and are released after PV.
+//
+// Exponentials: ex2.approx on the MUFU unit, except one column pair in four of every full
+// exact tile. Those use 2^x = 2^floor(x) * p(x - floor(x)), where p is a cubic minimax fit of 2^f
+// on [0, 1) (max relative error 8.6e-5, far below the bf16 rounding of P), evaluated with
+// packed f32x2 FMAs. That moves part of the exponential work from MUFU to the FMA pipe.
 //
 // Every mbarrier wait is bounded (sol::mbar_wait). On expiry the CTA records SOL_ETIMEOUT in the
 // workspace, the other roles stop at their next wait, in-flight copies and MMAs are drained, and
-// TMEM is freed before the kernel returns.
+// TMEM is freed before the kernel returns. The softmax groups leave the tile loop together
+// (a named-barrier OR vote), so no warp is ever left waiting at a named barrier.
 #include <cmath>
 
 #include "device_common.cuh"
@@ -35,35 +45,44 @@ namespace sol {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kSoftmaxWarp0 = 4;
+constexpr int kThreads = 320;
+constexpr int kSoftmaxWarp0 = 2;
+constexpr int kSoftmaxThreads = 256;
 constexpr int kRows = 128;  // B_q = B_k
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
 constexpr float kRescaleThreshold = 8.0f;  // lazy rescale: only when the row max grows by > 2^8
+constexpr uint32_t kBarSoftmax = 1;       // named barrier of the 256 softmax threads
+
+// cubic minimax fit of 2^f on [0, 1] with p(0) = 1 (relative error <= 8.6e-5)
+constexpr float kExpC1 = 0.69511664f, kExpC2 = 0.22764498f, kExpC3 = 0.07706724f;
 
 template <int D>
 struct TcCfg {
   static constexpr int NCHUNK = D / 64;                 // 128-byte swizzle atoms per row
   static constexpr int CHUNK_BYTES = kRows * 128;       // 128 rows x 128 B
   static constexpr int TILE_BYTES = NCHUNK * CHUNK_BYTES;
-  static constexpr int NSTAGE = (D == 128) ? 2 : 4;     // K/V ring depth
+  static constexpr int NK = (D == 128) ? 3 : 4;         // K ring depth
+  static constexpr int NV = (D == 128) ? 2 : 4;         // V ring depth
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + TILE_BYTES;
-  static constexpr int OFF_V = OFF_K + NSTAGE * TILE_BYTES;
-  static constexpr int OFF_SBAR = OFF_V + NSTAGE * TILE_BYTES;            // float[kMaxKeyBlocks]
+  static constexpr int OFF_V = OFF_K + NK * TILE_BYTES;
+  static constexpr int OFF_SBAR = OFF_V + NV * TILE_BYTES;                // float[kMaxKeyBlocks]
   static constexpr int OFF_KLIST = OFF_SBAR + kMaxKeyBlocks * 4;          // u16[kMaxKeyBlocks]
   static constexpr int OFF_BITS = OFF_KLIST + kMaxKeyBlocks * 2;          // u32[kMaxKeyBlocks/32]
   static constexpr int OFF_CLIST = OFF_BITS + kMaxKeyBlocks / 8;          // u16[kMaxKeyBlocks/128]
-  static constexpr int OFF_QBAR = OFF_CLIST + (kMaxKeyBlocks / 128) * 2;  // float[D] means + float[128] partials
-  static constexpr int OFF_RED = OFF_QBAR + (D + kRows) * 4;              // float[8]
+  static constexpr int OFF_QBAR = OFF_CLIST + (kMaxKeyBlocks / 128) * 2;  // float[D] + float[256] partials
+  static constexpr int OFF_XMAX = OFF_QBAR + (D + kSoftmaxThreads) * 4;   // float[2 buf][2 grp][128 rows]
+  static constexpr int OFF_LSUM = OFF_XMAX + 2 * 2 * kRows * 4;           // float[2 grp][128 rows]
+  static constexpr int OFF_RED = OFF_LSUM + 2 * kRows * 4;                // float[8]
   static constexpr int OFF_MISC = OFF_RED + 32;                           // int[8]
   static constexpr int OFF_BAR = OFF_MISC + 32;                           // mbarriers
-  // q_full, k_full[NSTAGE], v_full[NSTAGE], kv_empty[NSTAGE], s_full[2], p_full[2],
+  // q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2], p_full[2],
   // o_done, o_final, list_ready, drain
-  static constexpr int NBAR = 1 + 3 * NSTAGE + 2 + 2 + 4;
+  static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 2 + 2 + 4;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;  // + slack to align the base to 1024 B
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 struct TcParams {
@@ -83,6 +102,28 @@ struct TcParams {
 
 enum MiscSlot : int { MISC_UNIT = 0, MISC_NK = 1, MISC_NC = 2, MISC_ABORT = 3, MISC_LAST = 4 };
 
+// 2^x for a pair, on the FMA pipe: floor by a round-down add of 1.5*2^23, cubic on the fraction,
+// exponent added to the bit pattern. x must lie in [-126, 126].
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  const float2 t = __fadd2_rd(x, make_float2(12582912.0f, 12582912.0f));  // mantissa of t = floor(x)
+  const float2 j = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = __fadd2_rn(x, make_float2(-j.x, -j.y));                // in [0, 1)
+  float2 q = __ffma2_rn(f, make_float2(kExpC3, kExpC3), make_float2(kExpC2, kExpC2));
+  q = __ffma2_rn(f, q, make_float2(kExpC1, kExpC1));
+  q = __ffma2_rn(f, q, make_float2(1.0f, 1.0f));
+  const uint32_t ex = __float_as_uint(t.x) << 23, ey = __float_as_uint(t.y) << 23;  // floor(x) << 23
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + ex), __uint_as_float(__float_as_uint(q.y) + ey));
+}
+
+__device__ __forceinline__ float max64(const float (&s)[64]) {
+  float m8[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m8[k] = s[k];
+#pragma unroll
+  for (int c = 8; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+  return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     sol_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -98,15 +139,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* s_bits = reinterpret_cast<uint32_t*>(smem + C::OFF_BITS);
   uint16_t* s_clist = reinterpret_cast<uint16_t*>(smem + C::OFF_CLIST);
   float* s_qbar = reinterpret_cast<float*>(smem + C::OFF_QBAR);
+  float* s_xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);
+  float* s_lsum = reinterpret_cast<float*>(smem + C::OFF_LSUM);
   float* s_red = reinterpret_cast<float*>(smem + C::OFF_RED);
   volatile int* s_misc = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
   volatile int* s_abort = s_misc + MISC_ABORT;
 
   const uint32_t bar_q = sb + C::OFF_BAR;
   const uint32_t bar_kfull = bar_q + 8;
-  const uint32_t bar_vfull = bar_kfull + 8 * C::NSTAGE;
-  const uint32_t bar_kvempty = bar_vfull + 8 * C::NSTAGE;
-  const uint32_t bar_sfull = bar_kvempty + 8 * C::NSTAGE;
+  const uint32_t bar_kempty = bar_kfull + 8 * C::NK;
+  const uint32_t bar_vfull = bar_kempty + 8 * C::NK;
+  const uint32_t bar_vempty = bar_vfull + 8 * C::NV;
+  const uint32_t bar_sfull = bar_vempty + 8 * C::NV;
   const uint32_t bar_pfull = bar_sfull + 16;
   const uint32_t bar_odone = bar_pfull + 16;
   const uint32_t bar_ofinal = bar_odone + 8;
@@ -118,14 +162,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     mbar_init(bar_q, 1);
-    for (int s = 0; s < C::NSTAGE; ++s) {
+    for (int s = 0; s < C::NK; ++s) {
       mbar_init(bar_kfull + 8 * s, 1);
+      mbar_init(bar_kempty + 8 * s, 1);
+    }
+    for (int s = 0; s < C::NV; ++s) {
       mbar_init(bar_vfull + 8 * s, 1);
-      mbar_init(bar_kvempty + 8 * s, 1);
+      mbar_init(bar_vempty + 8 * s, 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_sfull + 8 * b, 1);
-      mbar_init(bar_pfull + 8 * b, kRows);
+      mbar_init(bar_pfull + 8 * b, kSoftmaxThreads);
     }
     mbar_init(bar_odone, 1);
     mbar_init(bar_ofinal, 1);
@@ -152,14 +199,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint32_t tile_base = 0;  // tiles processed by this CTA before the current unit (all roles agree)
   uint32_t unit_iter = 0;  // units processed by this CTA before the current one
-  // producer bookkeeping for the final drain: last load number armed on each stage, +1 (0 = none)
-  uint32_t armed[C::NSTAGE];  // 1 + use index of the last load armed on each stage (0 = none)
-  bool k_dropped[C::NSTAGE];
+  // producer bookkeeping for the final drain: 1 + use index of the last load armed per stage
+  uint32_t k_armed[C::NK], v_armed[C::NV];
 #pragma unroll
-  for (int s = 0; s < C::NSTAGE; ++s) {
-    armed[s] = 0;
-    k_dropped[s] = false;
-  }
+  for (int s = 0; s < C::NK; ++s) k_armed[s] = 0;
+#pragma unroll
+  for (int s = 0; s < C::NV; ++s) v_armed[s] = 0;
   bool mma_issued = false;
 
   for (;;) {
@@ -181,33 +226,50 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_PRODUCER);
         if (w == WAIT_OK) {
           const int nk = s_misc[MISC_NK], T = nk + s_misc[MISC_NC];
-          for (int t = 0; t < T; ++t) {
-            const uint32_t r = tile_base + t;
-            const int s = static_cast<int>(r % C::NSTAGE);
-            if (r >= static_cast<uint32_t>(C::NSTAGE)) {
-              w = mbar_wait(bar_kvempty + 8 * s, ((r / C::NSTAGE) - 1u) & 1u, s_abort, limit);
-              if (w != WAIT_OK) {
-                if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_PRODUCER);
-                break;
+          // K runs one tile ahead of V: K_0, K_1, V_0, K_2, V_1, ...
+          for (int t = 0; t <= T; ++t) {
+            if (t < T) {
+              const uint32_t g = tile_base + t;
+              const int s = static_cast<int>(g % C::NK);
+              if (g >= static_cast<uint32_t>(C::NK)) {
+                w = mbar_wait(bar_kempty + 8 * s, ((g / C::NK) - 1u) & 1u, s_abort, limit);
+                if (w != WAIT_OK) {
+                  if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_PRODUCER);
+                  break;
+                }
+              }
+              const bool exact = t < nk;
+              const void* mk = exact ? static_cast<const void*>(&tmK) : static_cast<const void*>(&tmKb);
+              const int y = (exact ? static_cast<int>(s_klist[t]) : static_cast<int>(s_clist[t - nk])) * kRows;
+              const bool drop = p.drop_one_load && blockIdx.x == 0 && unit_iter == 0 && t == 0;
+              if (!drop) {
+                mbar_arrive_expect_tx(bar_kfull + 8 * s, C::TILE_BYTES);
+                for (int c = 0; c < C::NCHUNK; ++c)
+                  tma_load_3d(sb + C::OFF_K + s * C::TILE_BYTES + c * C::CHUNK_BYTES, mk, bar_kfull + 8 * s, c * 64,
+                              y, bh);
+                k_armed[s] = g / C::NK + 1u;
               }
             }
-            const bool exact = t < nk;
-            const void* mk = exact ? static_cast<const void*>(&tmK) : static_cast<const void*>(&tmKb);
-            const void* mv = exact ? static_cast<const void*>(&tmV) : static_cast<const void*>(&tmVb);
-            const int y = (exact ? static_cast<int>(s_klist[t]) : static_cast<int>(s_clist[t - nk])) * kRows;
-            const bool drop = p.drop_one_load && blockIdx.x == 0 && unit_iter == 0 && t == 0;
-            if (!drop) {
-              mbar_arrive_expect_tx(bar_kfull + 8 * s, C::TILE_BYTES);
+            if (t >= 1) {
+              const int tp = t - 1;
+              const uint32_t g = tile_base + tp;
+              const int s = static_cast<int>(g % C::NV);
+              if (g >= static_cast<uint32_t>(C::NV)) {
+                w = mbar_wait(bar_vempty + 8 * s, ((g / C::NV) - 1u) & 1u, s_abort, limit);
+                if (w != WAIT_OK) {
+                  if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_PRODUCER);
+                  break;
+                }
+              }
+              const bool exact = tp < nk;
+              const void* mv = exact ? static_cast<const void*>(&tmV) : static_cast<const void*>(&tmVb);
+              const int y = (exact ? static_cast<int>(s_klist[tp]) : static_cast<int>(s_clist[tp - nk])) * kRows;
+              mbar_arrive_expect_tx(bar_vfull + 8 * s, C::TILE_BYTES);
               for (int c = 0; c < C::NCHUNK; ++c)
-                tma_load_3d(sb + C::OFF_K + s * C::TILE_BYTES + c * C::CHUNK_BYTES, mk, bar_kfull + 8 * s, c * 64,
+                tma_load_3d(sb + C::OFF_V + s * C::TILE_BYTES + c * C::CHUNK_BYTES, mv, bar_vfull + 8 * s, c * 64,
                             y, bh);
+              v_armed[s] = g / C::NV + 1u;
             }
-            mbar_arrive_expect_tx(bar_vfull + 8 * s, C::TILE_BYTES);
-            for (int c = 0; c < C::NCHUNK; ++c)
-              tma_load_3d(sb + C::OFF_V + s * C::TILE_BYTES + c * C::CHUNK_BYTES, mv, bar_vfull + 8 * s, c * 64, y,
-                          bh);
-            armed[s] = r / C::NSTAGE + 1u;
-            k_dropped[s] = drop;
           }
         }
       }
@@ -226,9 +288,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int t = 0; t <= T && ok; ++t) {
             if (t < T) {
               const uint32_t g = tile_base + t;
-              const int s = static_cast<int>(g % C::NSTAGE);
+              const int s = static_cast<int>(g % C::NK);
               const uint32_t b = g & 1u;
-              w = mbar_wait(bar_kfull + 8 * s, (g / C::NSTAGE) & 1u, s_abort, limit);
+              w = mbar_wait(bar_kfull + 8 * s, (g / C::NK) & 1u, s_abort, limit);
               if (w != WAIT_OK) {
                 if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_MMA);
                 ok = false;
@@ -244,15 +306,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               mma_issued = true;
               tc_commit(bar_sfull + 8 * b);
+              tc_commit(bar_kempty + 8 * s);
             }
             if (t >= 1) {
               // O += P V for the previous tile
               const int tp = t - 1;
               const uint32_t g = tile_base + tp;
-              const int s = static_cast<int>(g % C::NSTAGE);
+              const int s = static_cast<int>(g % C::NV);
               const uint32_t b = g & 1u;
               w = mbar_wait(bar_pfull + 8 * b, (g >> 1) & 1u, s_abort, limit);
-              if (w == WAIT_OK) w = mbar_wait(bar_vfull + 8 * s, (g / C::NSTAGE) & 1u, s_abort, limit);
+              if (w == WAIT_OK) w = mbar_wait(bar_vfull + 8 * s, (g / C::NV) & 1u, s_abort, limit);
               if (w != WAIT_OK) {
                 if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_MMA);
                 ok = false;
@@ -266,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_bf16_ts(tmem + kColO, p_col + kk * 8, smem_desc_sw128(v_addr + kk * 2048, C::CHUNK_BYTES, 1024),
                             idesc_pv, (tp > 0 || kk > 0) ? 1u : 0u);
               }
-              tc_commit(bar_kvempty + 8 * s);
+              tc_commit(bar_vempty + 8 * s);
               tc_commit(bar_odone);
             }
           }
@@ -275,21 +338,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (warp >= kSoftmaxWarp0) {
       // ------------------------------------------------------------------ router + softmax + epilogue
-      const int row = tid - kSoftmaxWarp0 * 32;  // 0..127, TMEM lane
-      const int wq = warp - kSoftmaxWarp0;       // TMEM lane quarter
+      const int st = tid - kSoftmaxWarp0 * 32;  // 0..255
+      const int grp = st >> 7;                  // column half: warps 2..5 -> 0, warps 6..9 -> 1
+      const int sw = st >> 5;                   // softmax warp 0..7
+      const int wq = (warp & 3);                // TMEM lane quarter this warp may access
+      const int row = wq * 32 + lane;           // query row = TMEM lane
       const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
       const int m_i = min(kRows, p.L - qb * kRows);
       const int nkb = p.nkb;
-      bool alive = true;
 
       int w = mbar_wait(bar_q, uphase, s_abort, limit);
       if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_ROUTER);
-      alive = !named_barrier_or(1, kRows, w != WAIT_OK);  // identical in all 128 threads
+      bool alive = !named_barrier_or(kBarSoftmax, kSoftmaxThreads, w != WAIT_OK);  // same in all 256
 
       // (1a) q_bar = mean of the valid query rows, read from the swizzled Q tile
       {
-        constexpr int TPC = kRows / D;  // threads per column: 1 (D=128) or 2 (D=64)
-        const int c = row % D, part = row / D;
+        constexpr int TPC = kSoftmaxThreads / D;  // threads per column: 2 (D=128) or 4 (D=64)
+        const int c = st % D, part = st / D;
         const uint8_t* qt = smem + C::OFF_Q + (c >> 6) * C::CHUNK_BYTES;
         const int cw = c & 63;
         float acc = 0.f;
@@ -299,18 +364,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             acc += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(qt + off));
           }
         }
-        s_qbar[D + row] = acc;
-        named_barrier_sync(1, kRows);
-        if (row < D) {
+        s_qbar[D + st] = acc;
+        named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
+        if (st < D) {
           float s = 0.f;
 #pragma unroll
-          for (int k = 0; k < TPC; ++k) s += s_qbar[D + row + k * D];
-          s_qbar[row] = s / static_cast<float>(m_i);
+          for (int k = 0; k < TPC; ++k) s += s_qbar[D + st + k * D];
+          s_qbar[st] = s / static_cast<float>(m_i);
         }
-        named_barrier_sync(1, kRows);
+        named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
       }
 
-      // (1b) proxy scores s_bar_j (shared memory only) and their max
+      // (1b) proxy scores s_bar_j (shared memory only) and their max; 8 warps, 4 rows in flight each
       {
         constexpr int DPL = D / 32;
         float qv[DPL];
@@ -318,11 +383,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < DPL; ++k) qv[k] = s_qbar[lane * DPL + k];
         const float* kb = p.kbar + static_cast<size_t>(bh) * nkb * D + lane * DPL;
         float wmax = -INFINITY;
-        for (int j0 = wq; j0 < nkb; j0 += 16) {
+        for (int j0 = sw; j0 < nkb; j0 += 32) {
           float dot[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int j = j0 + 4 * u;
+            const int j = j0 + 8 * u;
             dot[u] = 0.f;
             if (j < nkb) {
               const float* src = kb + static_cast<size_t>(j) * D;
@@ -342,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int j = j0 + 4 * u;
+            const int j = j0 + 8 * u;
             if (j < nkb) {
               const float s = dot[u] * p.inv_sqrt_d;
               if (lane == 0) s_sbar[j] = s;
@@ -350,13 +415,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (lane == 0) s_red[wq] = wmax;
-        named_barrier_sync(1, kRows);
+        if (lane == 0) s_red[sw] = wmax;
+        named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
       }
 
-      // (1c) keep bits, kept list, pooled-tile list (warp 0 of the group)
-      if (wq == 0) {
-        const float M = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
+      // (1c) keep bits, kept list, pooled-tile list (softmax warp 0)
+      if (sw == 0) {
+        float M = s_red[0];
+#pragma unroll
+        for (int k = 1; k < 8; ++k) M = fmaxf(M, s_red[k]);
         const float thr = M - p.tau[bh % p.H];
         int nk = 0;
         for (int base = 0; base < nkb; base += 32) {
@@ -391,52 +458,70 @@ __global__ void __launch_bounds__(kThreads, 1)
           atomicAdd(&p.ws[WS_COUNTS + bh], static_cast<uint32_t>(nk));
         }
       }
-      named_barrier_sync(1, kRows);
-      if (row == 0 && alive) mbar_arrive(bar_list);
+      named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
+      if (st == 0 && alive) mbar_arrive(bar_list);
       if (p.kept_mask != nullptr) {
         uint8_t* mrow = p.kept_mask + (static_cast<size_t>(bh) * p.nqb + qb) * nkb;
-        for (int j = row; j < nkb; j += kRows) mrow[j] = static_cast<uint8_t>((s_bits[j >> 5] >> (j & 31)) & 1u);
+        for (int j = st; j < nkb; j += kSoftmaxThreads)
+          mrow[j] = static_cast<uint8_t>((s_bits[j >> 5] >> (j & 31)) & 1u);
       }
 
-      // (2)+(3) online softmax over kept tiles, then pooled tiles
+      // (2)+(3) online softmax over kept tiles, then pooled tiles; this thread: row `row`,
+      // score columns [64 grp, 64 grp + 64)
       const int nk = s_misc[MISC_NK];
       const int T = alive ? nk + s_misc[MISC_NC] : 0;
+      const float sl2 = p.sl2;
       float m_run = -INFINITY, l_run = 0.f;
+      bool bad = false;  // a wait of this warp failed inside the tile loop
       for (int t = 0; t < T; ++t) {
         const uint32_t g = tile_base + t;
         const uint32_t b = g & 1u;
         w = mbar_wait(bar_sfull + 8 * b, (g >> 1) & 1u, s_abort, limit);
         if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_SOFTMAX);
-        if (!__all_sync(0xffffffffu, w == WAIT_OK)) {  // leave as a whole warp (tcgen05.ld is warp-wide)
+        const bool ok = __all_sync(0xffffffffu, w == WAIT_OK) && !bad;
+        float s[64];
+        float mx = -INFINITY;
+        const bool exact = t < nk;
+        const int j = exact ? static_cast<int>(s_klist[t]) : 0;
+        const bool full = exact && (j != nkb - 1 || p.last_n == kRows);
+        if (ok) {
+          tc_fence_after();
+          uint32_t raw[64];
+          tmem_ld_x64(tmem + lane_base + (b ? kColS1 : kColS0) + grp * 64, raw);
+#pragma unroll
+          for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(raw[c]);
+          if (full) {
+            mx = max64(s) * sl2;  // sl2 > 0: the max of the scaled scores
+          } else {
+            if (exact) {
+              const int valid = p.last_n - grp * 64;  // valid columns in this half
+#pragma unroll
+              for (int c = 0; c < 64; ++c) s[c] = (c < valid) ? s[c] * sl2 : -INFINITY;
+            } else {
+              const int cc = s_clist[t - nk];
+              const int valid = min(kRows, nkb - cc * kRows) - grp * 64;
+              const int nwords = (nkb + 31) / 32;
+              const uint32_t kw0 = (cc * 4 + grp * 2 < nwords) ? s_bits[cc * 4 + grp * 2] : 0u;
+              const uint32_t kw1 = (cc * 4 + grp * 2 + 1 < nwords) ? s_bits[cc * 4 + grp * 2 + 1] : 0u;
+              const int last_col = nkb - 1 - cc * kRows - grp * 64;  // column of the ragged last block, if here
+#pragma unroll
+              for (int c = 0; c < 64; ++c) {
+                const uint32_t kw = c < 32 ? kw0 : kw1;
+                const bool skipped = c < valid && !((kw >> (c & 31)) & 1u);
+                const float off = (c == last_col) ? p.log2_last_n : 7.0f;  // log2(n_j)
+                s[c] = skipped ? fmaf(s[c], sl2, off) : -INFINITY;
+              }
+            }
+            mx = max64(s);
+          }
+        }
+        // exchange the half-row maxima; the vote makes every softmax thread leave together
+        s_xmax[(b * 2 + grp) * kRows + row] = mx;
+        if (named_barrier_or(kBarSoftmax, kSoftmaxThreads, !ok)) {
           alive = false;
           break;
         }
-        tc_fence_after();
-        uint32_t sraw[128];
-        tmem_ld_x128(tmem + lane_base + (b ? kColS1 : kColS0), sraw);
-        float x[128];
-        if (t < nk) {
-          const int j = s_klist[t];
-          const int valid = (j == nkb - 1) ? p.last_n : kRows;
-#pragma unroll
-          for (int c = 0; c < 128; ++c) x[c] = (c < valid) ? __uint_as_float(sraw[c]) * p.sl2 : -INFINITY;
-        } else {
-          const int cc = s_clist[t - nk];
-          const int valid = min(kRows, nkb - cc * kRows);
-          uint32_t kw[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) kw[q] = (cc * 4 + q < (nkb + 31) / 32) ? s_bits[cc * 4 + q] : 0u;
-          const bool has_last = (cc * kRows + valid == nkb);
-#pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const bool skipped = c < valid && !((kw[c >> 5] >> (c & 31)) & 1u);
-            const float off = (has_last && c == valid - 1) ? p.log2_last_n : 7.0f;  // log2(n_j)
-            x[c] = skipped ? fmaf(__uint_as_float(sraw[c]), p.sl2, off) : -INFINITY;
-          }
-        }
-        float mt = x[0];
-#pragma unroll
-        for (int c = 1; c < 128; ++c) mt = fmaxf(mt, x[c]);
+        const float mt = fmaxf(s_xmax[(b * 2 + 0) * kRows + row], s_xmax[(b * 2 + 1) * kRows + row]);
         float m_new = m_run, alpha = 1.f;
         bool need = false;
         if (t == 0) {
@@ -446,62 +531,83 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_new = mt;
           alpha = ex2_approx(m_run - mt);
         }
-        uint32_t pk[64];
-        float rs = 0.f;
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float p0 = ex2_approx(x[2 * c] - m_new);
-          const float p1 = ex2_approx(x[2 * c + 1] - m_new);
-          rs += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
-        }
-        l_run = fmaf(l_run, alpha, rs);
         m_run = m_new;
+        uint32_t pk[32];
+        float2 rs0 = make_float2(0.f, 0.f), rs1 = make_float2(0.f, 0.f);
+        if (full) {
+          const float2 scale2 = make_float2(sl2, sl2);
+          const float2 negm2 = make_float2(-m_new, -m_new);
+#pragma unroll
+          for (int c2 = 0; c2 < 32; ++c2) {
+            const float2 x2 = __ffma2_rn(make_float2(s[2 * c2], s[2 * c2 + 1]), scale2, negm2);
+            float2 e2;
+            if ((c2 & 3) == 3) {
+              e2 = exp2_poly2(make_float2(fmaxf(x2.x, -126.f), fmaxf(x2.y, -126.f)));
+            } else {
+              e2 = make_float2(ex2_approx(x2.x), ex2_approx(x2.y));
+            }
+            pk[c2] = pack_bf16x2(e2.x, e2.y);
+            const float2 r2 = make_float2(__uint_as_float(pk[c2] << 16), __uint_as_float(pk[c2] & 0xffff0000u));
+            if (c2 & 1) rs1 = __fadd2_rn(rs1, r2); else rs0 = __fadd2_rn(rs0, r2);
+          }
+        } else {
+#pragma unroll
+          for (int c2 = 0; c2 < 32; ++c2) {
+            const float e0 = ex2_approx(s[2 * c2] - m_new);
+            const float e1 = ex2_approx(s[2 * c2 + 1] - m_new);
+            pk[c2] = pack_bf16x2(e0, e1);
+            const float2 r2 = make_float2(__uint_as_float(pk[c2] << 16), __uint_as_float(pk[c2] & 0xffff0000u));
+            if (c2 & 1) rs1 = __fadd2_rn(rs1, r2); else rs0 = __fadd2_rn(rs0, r2);
+          }
+        }
+        // the row sum takes the same bf16-rounded weights the PV MMA uses
+        l_run = fmaf(l_run, alpha, (rs0.x + rs0.y) + (rs1.x + rs1.y));
         if (__any_sync(0xffffffffu, need)) {
-          // rescale O after the previous tile's PV has landed
+          // rescale this group's half of O after the previous tile's PV has landed
           w = mbar_wait(bar_odone, (g - 1u) & 1u, s_abort, limit);
           if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_SOFTMAX);
-          if (!__all_sync(0xffffffffu, w == WAIT_OK)) {
-            alive = false;
-            break;
-          }
-          tc_fence_after();
+          if (__all_sync(0xffffffffu, w == WAIT_OK)) {
+            tc_fence_after();
 #pragma unroll
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t o[32];
-            tmem_ld_x32(tmem + lane_base + kColO + ch * 32, o);
+            for (int ch = 0; ch < D / 64; ++ch) {
+              uint32_t o[32];
+              const uint32_t oc = tmem + lane_base + kColO + grp * (D / 2) + ch * 32;
+              tmem_ld_x32(oc, o);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st_x32(tmem + lane_base + kColO + ch * 32, o);
+              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+              tmem_st_x32(oc, o);
+            }
+          } else {
+            bad = true;  // leave at the next vote; P is still published so nothing else blocks
           }
         }
-        uint32_t pk0[32], pk1[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          pk0[c] = pk[c];
-          pk1[c] = pk[32 + c];
-        }
-        const uint32_t pcol = tmem + lane_base + (b ? kColP1 : kColP0);
-        tmem_st_x32(pcol, pk0);
-        tmem_st_x32(pcol + 32, pk1);
+        tmem_st_x32(tmem + lane_base + (b ? kColP1 : kColP0) + grp * 32, pk);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar_pfull + 8 * b);
       }
 
-      // (4) epilogue: O / l -> bf16
-      if (alive && T > 0) {
-        w = mbar_wait(bar_ofinal, uphase, s_abort, limit);
-        if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_SOFTMAX);
-        if (__all_sync(0xffffffffu, w == WAIT_OK)) {
+      // (4) epilogue: combine the two half-row sums, O / l -> bf16, each group stores its columns
+      {
+        bool ok = alive && !bad && T > 0;
+        if (ok) {
+          w = mbar_wait(bar_ofinal, uphase, s_abort, limit);
+          if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_SOFTMAX);
+          ok = __all_sync(0xffffffffu, w == WAIT_OK);
+        }
+        // every softmax thread reaches this barrier: the tile loop is left by all of them together
+        s_lsum[grp * kRows + row] = l_run;
+        const bool any_bad = named_barrier_or(kBarSoftmax, kSoftmaxThreads, !ok);
+        if (!any_bad) {
           tc_fence_after();
-          const float inv = 1.f / l_run;
+          const float inv = 1.f / (s_lsum[row] + s_lsum[kRows + row]);
           const bool store = row < m_i;
-          __nv_bfloat16* dst = p.O + (static_cast<size_t>(bh) * p.L + static_cast<size_t>(qb) * kRows + row) * D;
+          __nv_bfloat16* dst = p.O + (static_cast<size_t>(bh) * p.L + static_cast<size_t>(qb) * kRows + row) * D +
+                               grp * (D / 2);
 #pragma unroll
-          for (int ch = 0; ch < D / 32; ++ch) {
+          for (int ch = 0; ch < D / 64; ++ch) {
             uint32_t o[32];
-            tmem_ld_x32(tmem + lane_base + kColO + ch * 32, o);
+            tmem_ld_x32(tmem + lane_base + kColO + grp * (D / 2) + ch * 32, o);
             uint32_t pkd[16];
 #pragma unroll
             for (int c = 0; c < 16; ++c)
@@ -529,12 +635,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_wait(bar_drain, 0, nullptr, limit);
   }
   if (warp == 0 && lane == 0) {
-    for (int s = 0; s < C::NSTAGE; ++s) {
-      if (armed[s] == 0) continue;
-      const uint32_t use = armed[s] - 1u;
-      if (!k_dropped[s]) mbar_wait(bar_kfull + 8 * s, use & 1u, nullptr, limit);
-      mbar_wait(bar_vfull + 8 * s, use & 1u, nullptr, limit);
-    }
+    for (int s = 0; s < C::NK; ++s)
+      if (k_armed[s]) mbar_wait(bar_kfull + 8 * s, (k_armed[s] - 1u) & 1u, nullptr, limit);
+    for (int s = 0; s < C::NV; ++s)
+      if (v_armed[s]) mbar_wait(bar_vfull + 8 * s, (v_armed[s] - 1u) & 1u, nullptr, limit);
     if (unit_iter > 0) mbar_wait(bar_q, (unit_iter - 1u) & 1u, nullptr, limit);
   }
   tc_fence_before();
