@@ -116,12 +116,16 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
 }
 
 __device__ __forceinline__ float max64(const float (&s)[64]) {
-  float m8[8];
+  // four independent chains of three-input max over the 64 values
+  float m[4] = {fmax3(s[0], s[1], s[2]), fmax3(s[3], s[4], s[5]), fmax3(s[6], s[7], s[8]), fmax3(s[9], s[10], s[11])};
 #pragma unroll
-  for (int k = 0; k < 8; ++k) m8[k] = s[k];
+  for (int c = 12; c < 60; c += 8) {
 #pragma unroll
-  for (int c = 8; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
-  return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+    for (int k = 0; k < 4; ++k) m[k] = fmax3(m[k], s[c + 2 * k], s[c + 2 * k + 1]);
+  }
+  m[0] = fmax3(m[0], s[60], s[61]);
+  m[1] = fmax3(m[1], s[62], s[63]);
+  return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
 
 template <int D>
@@ -533,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         m_run = m_new;
         uint32_t pk[32];
-        float2 rs0 = make_float2(0.f, 0.f), rs1 = make_float2(0.f, 0.f);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};  // row sum of the bf16-rounded weights, 4 chains
         if (full) {
           const float2 scale2 = make_float2(sl2, sl2);
           const float2 negm2 = make_float2(-m_new, -m_new);
@@ -547,8 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               e2 = make_float2(ex2_approx(x2.x), ex2_approx(x2.y));
             }
             pk[c2] = pack_bf16x2(e2.x, e2.y);
-            const float2 r2 = make_float2(__uint_as_float(pk[c2] << 16), __uint_as_float(pk[c2] & 0xffff0000u));
-            if (c2 & 1) rs1 = __fadd2_rn(rs1, r2); else rs0 = __fadd2_rn(rs0, r2);
+            acc[c2 & 3] = add_bf16x2(acc[c2 & 3], pk[c2]);
           }
         } else {
 #pragma unroll
@@ -556,19 +559,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float e0 = ex2_approx(s[2 * c2] - m_new);
             const float e1 = ex2_approx(s[2 * c2 + 1] - m_new);
             pk[c2] = pack_bf16x2(e0, e1);
-            const float2 r2 = make_float2(__uint_as_float(pk[c2] << 16), __uint_as_float(pk[c2] & 0xffff0000u));
-            if (c2 & 1) rs1 = __fadd2_rn(rs1, r2); else rs0 = __fadd2_rn(rs0, r2);
+            acc[c2 & 3] = add_bf16x2(acc[c2 & 3], pk[c2]);
           }
         }
         // the row sum takes the same bf16-rounded weights the PV MMA uses
-        l_run = fmaf(l_run, alpha, (rs0.x + rs0.y) + (rs1.x + rs1.y));
+        l_run = fmaf(l_run, alpha, (acc[0] + acc[1]) + (acc[2] + acc[3]));
+        tmem_st_x32(tmem + lane_base + (b ? kColP1 : kColP0) + grp * 32, pk);
         if (__any_sync(0xffffffffu, need)) {
           // rescale this group's half of O after the previous tile's PV has landed
           w = mbar_wait(bar_odone, (g - 1u) & 1u, s_abort, limit);
           if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_SOFTMAX);
           if (__all_sync(0xffffffffu, w == WAIT_OK)) {
             tc_fence_after();
-#pragma unroll
+#pragma unroll 1
             for (int ch = 0; ch < D / 64; ++ch) {
               uint32_t o[32];
               const uint32_t oc = tmem + lane_base + kColO + grp * (D / 2) + ch * 32;
@@ -581,7 +584,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             bad = true;  // leave at the next vote; P is still published so nothing else blocks
           }
         }
-        tmem_st_x32(tmem + lane_base + (b ? kColP1 : kColP0) + grp * 32, pk);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar_pfull + 8 * b);
