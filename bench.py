@@ -63,6 +63,43 @@ def peaks():
     return {**FALLBACK_PEAKS, "bf16_tflops_sustained": FALLBACK_PEAKS["bf16_tflops"], "source": "fallback"}
 
 
+def reduce_max_over_ranks(x: float, world: int, device) -> float:
+    """MAX of a per-rank time over all ranks (the only collective; none on the data path)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def kernel_source_hash() -> str:
+    """First 16 hex digits of the sha256 of the tensor-core kernel's sources (as in profiles/)."""
+    import hashlib
+    csrc = os.path.join(ROOT, "block_sparse_attention_41_b200", "csrc")
+    data = b"".join(open(os.path.join(csrc, f), "rb").read() for f in ("fwd_tc.cu", "device_common.cuh"))
+    return hashlib.sha256(data).hexdigest()[:16]
+
+
+def captured_traffic(w, key):
+    """DRAM bytes per fwd launch from the committed ncu summary, or None when there is no capture
+    for this workload and density or the kernel source changed since it was taken."""
+    import re
+    path = os.path.join(ROOT, "profiles", f"sol_fwd_tc_kernel_{w.name}.md")
+    if not os.path.exists(path):
+        return None
+    m = re.search(r"```json\s*(\{.*?\})\s*```", open(path).read(), re.S)
+    if not m:
+        return None
+    rec = json.loads(m.group(1))
+    if rec.get("density") != key or rec.get("scaled_to_heads") != w.H:
+        return None
+    if rec.get("source_sha256_16") != kernel_source_hash():
+        return None
+    return rec.get("bytes_per_launch")
+
+
 def kept_tile_flops(kept_blocks: int, w) -> float:
     return 4.0 * w.block * w.block * w.d * kept_blocks
 
@@ -157,7 +194,7 @@ def run_reference(args, w):
         return 0
     key = args.density if args.density in density_keys(w) else density_keys(w)[0]
     tau = tau_for(w, key)
-    per_step = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    per_step = args.ref_budget or max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         oracle_sample(w, tau, per_step * 0.25, seed_offset=1)
     tiles, secs = 0, 0.0
@@ -220,11 +257,7 @@ def run_ours(args, w):
             dist.barrier()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max_over_ranks(x, world, dev)
 
     sa.load_library()
     Q, K, V = device_inputs(w, dev, torch)
@@ -344,13 +377,7 @@ def run_ours(args, w):
                "sample": f"{units} seeded query-block units of {w.name} at density {key} "
                          f"({secs:.1f} s of float64 oracle work, extrapolated per kept tile)"}
 
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(prof):
-        with open(prof) as f:
-            tr = json.load(f)
-        if tr.get("workload") == w.name and tr.get("density") == key:
-            traffic = tr.get("bytes_per_launch")
+    traffic = captured_traffic(w, key)
 
     if rank == 0:
         clocks = clk.summary()
@@ -401,6 +428,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-budget", type=float, default=0.0,
+                    help="reference arm: seconds of oracle work per step (default: fit a few minutes)")
     ap.add_argument("--heads", type=int, default=0,
                     help="profiling only: keep the first N heads of the workload (same seeds)")
     args = ap.parse_args()
