@@ -86,6 +86,38 @@ sol_status make_map(CUtensorMap* m, const void* base, int d, int rows, int BH) {
 
 bool size_ok(long long v, long long lim) { return v >= 1 && v <= lim; }
 
+// ---- workspace in the library's own device memory, for sol_attn_fwd_noalloc -------------------
+constexpr int kNoAllocMaxHeads = 4096;  // B * H
+constexpr size_t kNoAllocWords = static_cast<size_t>(sol::WS_COUNTS) + kNoAllocMaxHeads;
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+}  // namespace
+
+// One array per device that loads the library, alive until the process exits. In host code this
+// name is only a host-side handle: its device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) uint32_t g_noalloc_ws[kNoAllocWords];
+
+namespace {
+
+// Device address of g_noalloc_ws on the current device, looked up once per device.
+sol_status noalloc_workspace(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(SOL_EUNSUPPORTED, "device index %d beyond %d", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_ws);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static workspace)");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SOL_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -238,6 +270,26 @@ sol_status sol_attn_fwd(const void* Q, const void* K, const void* V, const float
     if (e != cudaSuccess) return cuda_fail(e, "fp32 forward launch");
   }
   return SOL_OK;
+}
+
+sol_status sol_attn_fwd_noalloc(const void* Q, const void* K, const void* V, const float* kbar, const float* vbar,
+                                const void* kbar_lp, const void* vbar_lp, const float* tau, sol_dtype dt, int B, int H,
+                                int L, int d, int block_q, int block_k, int n_force, void* O, uint8_t* kept_mask,
+                                float* density, void* stream) {
+  g_last_error.clear();
+  if (B < 1 || H < 1) return fail(SOL_EINVAL, "B and H must be positive (B=%d H=%d)", B, H);
+  if (static_cast<long long>(B) * H > kNoAllocMaxHeads)
+    return fail(SOL_EUNSUPPORTED, "B*H=%lld exceeds the %d heads the static workspace holds; use sol_attn_fwd",
+                static_cast<long long>(B) * H, kNoAllocMaxHeads);
+  void* ws = nullptr;
+  sol_status st = noalloc_workspace(&ws);
+  if (st != SOL_OK) return st;
+  // the array keeps the previous call's contents: clear all of it (counters and error word)
+  const size_t bytes = sizeof(uint32_t) * kNoAllocWords;
+  cudaError_t e = cudaMemsetAsync(ws, 0, bytes, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(static workspace)");
+  return sol_attn_fwd(Q, K, V, kbar, vbar, kbar_lp, vbar_lp, tau, dt, B, H, L, d, block_q, block_k, n_force, O,
+                      kept_mask, density, ws, bytes, stream);
 }
 
 sol_status sol_attn_check_device_error(void* workspace, void* stream) {

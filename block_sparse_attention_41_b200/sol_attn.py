@@ -29,6 +29,7 @@ EXPORTED = (
     "sol_attn_fwd",
     "sol_attn_check_device_error",
     "sol_attn_debug_drop_one_load",
+    "sol_attn_fwd_noalloc",
 )
 
 
@@ -65,6 +66,9 @@ def load_library() -> ctypes.CDLL:
     lib.sol_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, f32p, i32, i32, i32, i32, i32, i32, i32, i32,
                                  vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.sol_attn_fwd.restype = i32
+    lib.sol_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, f32p, i32, i32, i32, i32, i32, i32, i32, i32,
+                                         vp, vp, vp, vp]
+    lib.sol_attn_fwd_noalloc.restype = i32
     lib.sol_attn_check_device_error.argtypes = [vp, vp]
     lib.sol_attn_check_device_error.restype = i32
     lib.sol_attn_debug_drop_one_load.argtypes = [i32]
@@ -174,6 +178,30 @@ def sol_attn_fwd(Q, K, V, kbar, vbar, kbar_lp, vbar_lp, tau: Sequence[float], bl
         block_q, block_k, int(n_force), _ptr(O), _ptr(kept_mask), _ptr(density), _ptr(workspace),
         workspace.numel(), _stream(stream))
     _check(st, "sol_attn_fwd")
+    return O
+
+
+def sol_attn_fwd_noalloc(Q, K, V, kbar, vbar, kbar_lp, vbar_lp, tau: Sequence[float], block_q: int, block_k: int,
+                         n_force: int = 0, O=None, kept_mask=None, density=None, stream=None):
+    """sol_attn_fwd without a workspace argument: the library uses its own static device array
+    (B*H <= 4096; calls that overlap on the GPU race on it). For callers that cannot allocate
+    device memory; pass a preallocated `O` to allocate nothing here either."""
+    _need_cuda("Q", Q)
+    for n, t in (("K", K), ("V", V)):
+        _need_cuda(n, t, Q.dtype)
+    B, H, L, d = Q.shape
+    if K.shape != Q.shape or V.shape != Q.shape:
+        raise ValueError("Q, K and V must have the same shape [B, H, L, d]")
+    tau = [float(x) for x in tau]
+    if len(tau) != H:
+        raise ValueError(f"tau must hold H={H} values")
+    if O is None:
+        O = torch.empty_like(Q)
+    tau_c = (ctypes.c_float * H)(*tau)
+    st = load_library().sol_attn_fwd_noalloc(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(kbar), _ptr(vbar), _ptr(kbar_lp), _ptr(vbar_lp), tau_c, _dtype_code(Q), B, H,
+        L, d, block_q, block_k, int(n_force), _ptr(O), _ptr(kept_mask), _ptr(density), _stream(stream))
+    _check(st, "sol_attn_fwd_noalloc")
     return O
 
 

@@ -23,7 +23,8 @@
  *     padding; partial last blocks are masked inside the kernels), [B, H, N_kb, d] for pooled
  *     vectors, with N_kb = ceil(L / block_k) and N_qb = ceil(L / block_q).
  *   - Device pointers must be 16-byte aligned. All device memory and the stream belong to the
- *     caller; the library allocates nothing and keeps no global state.
+ *     caller; the library allocates nothing and keeps no global state (the one exception is the
+ *     static device array of sol_attn_fwd_noalloc, described there).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). Every call
  *     that launches work is asynchronous on that stream.
  *   - Arguments are validated on the host before any launch. Invalid ones return SOL_EINVAL,
@@ -113,6 +114,35 @@ sol_status sol_attn_fwd(const void* Q, const void* K, const void* V, const float
  * SOL_ETIMEOUT if any launch since the last check gave up on a bounded wait, after which that
  * launch's outputs are incomplete. Returns SOL_OK otherwise. */
 sol_status sol_attn_check_device_error(void* workspace, void* stream);
+
+/* The same fused forward for callers that cannot allocate device memory. There is no counterpart
+ * on the Sol-Attn pages; this is a deployment convenience of this library.
+ *
+ * Some callers cannot call cudaMalloc. Examples: a host framework whose caching allocator has
+ * already reserved the device memory and forbids foreign allocations; a plugin that must not
+ * trigger the implicit device synchronisation cudaMalloc/cudaFree can cause on a latency-critical
+ * path. Such callers cannot provide the workspace that sol_attn_fwd needs. This entry point takes
+ * the same arguments minus the workspace. It uses a 16,400-byte array in the library's own device
+ * memory instead: a file-scope static __device__ array, which every GPU that loads the library
+ * holds until the process exits.
+ *
+ *   limit      B * H <= 4096 (the array holds the counters of at most 4096 heads); larger
+ *              problems return SOL_EUNSUPPORTED without launching anything.
+ *   set-up     the first call on a device looks up the array's device address
+ *              (cudaGetSymbolAddress) with that device current, and caches it. Make that first
+ *              call before any stream capture.
+ *   sharing    every call on a device shares the one array. Each call clears it on `stream`
+ *              before launching, so calls on one stream are safe, but calls that overlap on the
+ *              GPU (different streams, no ordering) race on it.
+ *   errors     host-side errors as for sol_attn_fwd. The device error word of a bounded-wait
+ *              expiry is kept in the shared array and is not readable through this ABI. Use
+ *              sol_attn_fwd with a workspace when that status is needed.
+ * Calls no cudaMalloc, cudaFree or other allocating routine. */
+sol_status sol_attn_fwd_noalloc(const void* Q, const void* K, const void* V, const float* kbar,
+                                const float* vbar, const void* kbar_lp, const void* vbar_lp,
+                                const float* tau, sol_dtype dt, int B, int H, int L, int d,
+                                int block_q, int block_k, int n_force, void* O, uint8_t* kept_mask,
+                                float* density, void* stream);
 
 /* Test hook for the failure-detection path. mode 0 (default) = normal operation. mode 1 makes
  * the next sol_attn_fwd launch (SOL_BF16 path) skip one K-tile load, so the consumer's bounded

@@ -1,0 +1,86 @@
+"""The allocation-free forward entry point, sol_attn_fwd_noalloc, against sol_attn_fwd.
+
+Some callers cannot call cudaMalloc: a host framework whose allocator already owns the device
+memory, or a latency-critical caller that must avoid the device-wide synchronisation an
+allocation can cause. They cannot hand sol_attn_fwd a workspace, so the library offers this
+variant, which keeps its scratch counters in its own static device array. This file checks,
+through the C ABI, that two calls in a row give the same outputs as the workspace entry point
+within the parity tolerances, and that oversized problems are refused before any launch.
+It is collected last so that a run stopping at the first failure has run everything else first.
+"""
+import ctypes
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_41_b200 import sol_attn as sa
+from block_sparse_attention_41_b200.workloads import round_to_bf16
+
+pytestmark = pytest.mark.gpu
+
+TOL_MAX, TOL_MEAN = 2e-2, 2e-3   # bf16 parity tolerances used by the other GPU tests
+TOL_F32 = 1e-4
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from block_sparse_attention_41_b200 import build
+    build.build()
+    sa.load_library()
+
+
+def _inputs(B, H, L, d, dtype, seed):
+    rng = np.random.default_rng(seed)
+    t = np.arange(L)[:, None] / 40.0
+    c = np.arange(d)[None, :]
+    feat = np.where(c % 2 == 0, np.sin(t * (1 + c % 5)), np.cos(t * (1 + c % 3))) * 2.0
+    arrs = [rng.standard_normal((B, H, L, d)) + (feat if i < 2 else 0) for i in range(3)]
+    if dtype == torch.bfloat16:
+        arrs = [round_to_bf16(a) for a in arrs]
+    return [torch.from_numpy(np.asarray(a, dtype=np.float32)).to(dtype).cuda() for a in arrs]
+
+
+@pytest.mark.parametrize("dtype,L,d,block,tau", [
+    (torch.bfloat16, 3000, 128, 128, [0.0, 0.7, 2.5, math.inf]),
+    (torch.bfloat16, 1500, 64, 128, [0.4, 1.0, 1.5, 3.0]),
+    (torch.float32, 700, 64, 64, [0.3, 1.2, 2.0, math.inf]),
+])
+def test_noalloc_matches_workspace_entry_point_twice(dtype, L, d, block, tau):
+    B, H = 1, 4
+    Q, K, V = _inputs(B, H, L, d, dtype, seed=L + d)
+    kbar, vbar, klp, vlp = sa.sol_attn_pool(K, V, block)
+    nb = -(-L // block)
+    ref_mask = torch.empty((B, H, nb, nb), dtype=torch.uint8, device="cuda")
+    ref_dens = torch.empty((B, H), dtype=torch.float32, device="cuda")
+    ref = sa.sol_attn_fwd(Q, K, V, kbar, vbar, klp, vlp, tau, block, block, kept_mask=ref_mask, density=ref_dens)
+    torch.cuda.synchronize()
+    for _ in range(2):  # two calls in a row share (and must re-clear) the static array
+        O = torch.full_like(Q, float("nan"))
+        mask = torch.zeros_like(ref_mask)
+        dens = torch.zeros_like(ref_dens)
+        sa.sol_attn_fwd_noalloc(Q, K, V, kbar, vbar, klp, vlp, tau, block, block, O=O, kept_mask=mask,
+                                density=dens)
+        torch.cuda.synchronize()
+        err = (O.double() - ref.double()).abs()
+        if dtype == torch.float32:
+            assert float(err.max()) <= TOL_F32
+        else:
+            assert float(err.max()) <= TOL_MAX and float(err.mean()) <= TOL_MEAN
+        assert torch.equal(mask, ref_mask)
+        assert torch.allclose(dens, ref_dens, rtol=0, atol=1e-7)
+
+
+def test_noalloc_refuses_more_heads_than_the_static_array_holds():
+    lib = sa.load_library()
+    x = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
+    p = ctypes.c_void_p(x.data_ptr())
+    H = 4097
+    tau = (ctypes.c_float * H)(*([1.0] * H))
+    st = lib.sol_attn_fwd_noalloc(p, p, p, p, p, p, p, tau, sa.SOL_BF16, 1, H, 128, 128, 128, 128, 0, p, None,
+                                  None, None)
+    assert st == sa.SOL_EUNSUPPORTED
+    assert "4096" in lib.sol_attn_last_error().decode()
