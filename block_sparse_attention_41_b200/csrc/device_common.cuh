@@ -113,6 +113,12 @@ __device__ __forceinline__ bool named_barrier_or(uint32_t id, uint32_t nthreads,
 }
 
 // ---- TMA -------------------------------------------------------------------------------------
+// Order this thread's earlier generic-proxy accesses of shared memory before later async-proxy
+// accesses (TMA writes) of the same bytes.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }

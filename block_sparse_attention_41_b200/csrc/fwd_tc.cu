@@ -14,18 +14,25 @@
 //                 MMA/softmax pipeline and the same running max, sum and accumulator.
 //   4. epilogue : O / l -> bf16 -> global.
 //
-// Roles (320 threads): warp 0 = TMA producer, warp 1 = MMA issuer (also owns TMEM), warps 2..5
-// and 6..9 = two softmax groups. A warp may only touch TMEM lanes 32*(warp%4) .. +31, and any four
+// Roles (352 threads): warp 0 = TMA producer, warp 1 = PV issuer (also owns TMEM), warps 2..5
+// and 6..9 = two softmax groups, warp 10 = QK^T issuer. A tcgen05.mma blocks its issuing thread
+// for about as long as the tensor pipe takes to run it, so the two products are issued from two
+// threads: waiting for one tile's PV to finish (before its S buffer is refilled) never delays the
+// PV of the next tile. A warp may only touch TMEM lanes 32*(warp%4) .. +31, and any four
 // consecutive warps cover all four quarters, so thread (g, r) of softmax group g owns query
-// row r (TMEM lane r) and score columns [64g, 64g+64). The two halves exchange their row max
-// once per tile through shared memory. Both groups also do the routing and the epilogue. Units
-// come from an atomic counter in head-major order, so CTAs running at the same time share one
-// head's K/V in L2.
+// row r (TMEM lane r) and score columns [64g, 64g+64) of every tile.
 //
-// TMEM columns: S0 [0,128) S1 [128,256) O [256,256+D) P0 [384,448) P1 [448,512).
-// P has its own columns, separate from S, so the QK^T that refills S[b] never races the PV MMA
-// that reads P[b]. K tiles go round a 3-deep ring (d = 128) and are released as soon as their
-// QK^T completes. V tiles go round a 2-deep ring and are released after PV.
+// The two groups never synchronise inside the tile loop. Each keeps its own running max m_g and
+// sum l_g over its half of the key columns and accumulates its own output O_g = sum P_g V_g in
+// TMEM. That is the same softmax split into two partial sums over disjoint key sets; the
+// epilogue merges them once per unit with the usual rescale,
+//   O = (2^(m_0-m) O_0 + 2^(m_1-m) O_1) / (2^(m_0-m) l_0 + 2^(m_1-m) l_1),  m = max(m_0, m_1).
+//
+// TMEM columns: S0 [0,128) S1 [128,256) O_0 [256,256+D) O_1 [256+D,256+2D). Group g writes its
+// bf16 P over S columns [64g, 64g+32) of the buffer it has just read. S is double-buffered, so
+// the refill of a buffer (the QK^T of tile t+2, issued once the PV of tile t has completed) runs
+// while the softmax works on tile t+1. K tiles go round a 3-deep ring (d = 128) and are released
+// as soon as their QK^T completes; V tiles go round a 2-deep ring and are released after PV.
 //
 // Exponentials: ex2.approx on the MUFU unit, except one column pair in four of every full
 // exact tile. Those use 2^x = 2^floor(x) * p(x - floor(x)), where p is a cubic minimax fit of 2^f
@@ -34,8 +41,8 @@
 //
 // Every mbarrier wait is bounded (sol::mbar_wait). On expiry the CTA records SOL_ETIMEOUT in the
 // workspace, the other roles stop at their next wait, in-flight copies and MMAs are drained, and
-// TMEM is freed before the kernel returns. The softmax groups leave the tile loop together
-// (a named-barrier OR vote), so no warp is ever left waiting at a named barrier.
+// TMEM is freed before the kernel returns. Every softmax warp reaches the epilogue's named
+// barrier whether or not its tile loop ended early, so no warp is left waiting there.
 #include <cmath>
 
 #include "device_common.cuh"
@@ -45,12 +52,15 @@ namespace sol {
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kSoftmaxWarp0 = 2;
+constexpr int kQkWarp = 10;
 constexpr int kSoftmaxThreads = 256;
-constexpr int kRows = 128;  // B_q = B_k
+constexpr int kGroupWarps = 4;  // warps per softmax group
+constexpr int kRows = 128;      // B_q = B_k
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
+constexpr uint32_t kColS = 0;    // S buffer b at kColS + 128 b
+constexpr uint32_t kColO = 256;  // O_g at kColO + D g
 constexpr float kRescaleThreshold = 8.0f;  // lazy rescale: only when the row max grows by > 2^8
 constexpr uint32_t kBarSoftmax = 1;       // named barrier of the 256 softmax threads
 
@@ -72,17 +82,17 @@ struct TcCfg {
   static constexpr int OFF_BITS = OFF_KLIST + kMaxKeyBlocks * 2;          // u32[kMaxKeyBlocks/32]
   static constexpr int OFF_CLIST = OFF_BITS + kMaxKeyBlocks / 8;          // u16[kMaxKeyBlocks/128]
   static constexpr int OFF_QBAR = OFF_CLIST + (kMaxKeyBlocks / 128) * 2;  // float[D] + float[256] partials
-  static constexpr int OFF_XMAX = OFF_QBAR + (D + kSoftmaxThreads) * 4;   // float[2 buf][2 grp][128 rows]
-  static constexpr int OFF_LSUM = OFF_XMAX + 2 * 2 * kRows * 4;           // float[2 grp][128 rows]
-  static constexpr int OFF_RED = OFF_LSUM + 2 * kRows * 4;                // float[8]
+  static constexpr int OFF_ML = OFF_QBAR + (D + kSoftmaxThreads) * 4;     // float2[2 grp][128 rows]
+  static constexpr int OFF_RED = OFF_ML + 2 * kRows * 8;                  // float[8]
   static constexpr int OFF_MISC = OFF_RED + 32;                           // int[8]
   static constexpr int OFF_BAR = OFF_MISC + 32;                           // mbarriers
-  // q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2], p_full[2],
-  // o_done, o_final, list_ready, drain
-  static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 2 + 2 + 4;
+  // q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2], p_full[2 buf][2 grp],
+  // pv_done[2 buf], o_final, list_ready, drain[2 issuers]
+  static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 2 + 4 + 2 + 1 + 1 + 2;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;  // + slack to align the base to 1024 B
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(kColO + 2 * D <= kTmemCols, "TMEM budget");
 };
 
 struct TcParams {
@@ -137,14 +147,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
-
   float* s_sbar = reinterpret_cast<float*>(smem + C::OFF_SBAR);
   uint16_t* s_klist = reinterpret_cast<uint16_t*>(smem + C::OFF_KLIST);
   uint32_t* s_bits = reinterpret_cast<uint32_t*>(smem + C::OFF_BITS);
   uint16_t* s_clist = reinterpret_cast<uint16_t*>(smem + C::OFF_CLIST);
   float* s_qbar = reinterpret_cast<float*>(smem + C::OFF_QBAR);
-  float* s_xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);
-  float* s_lsum = reinterpret_cast<float*>(smem + C::OFF_LSUM);
+  float2* s_ml = reinterpret_cast<float2*>(smem + C::OFF_ML);
   float* s_red = reinterpret_cast<float*>(smem + C::OFF_RED);
   volatile int* s_misc = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
   volatile int* s_abort = s_misc + MISC_ABORT;
@@ -154,12 +162,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_kempty = bar_kfull + 8 * C::NK;
   const uint32_t bar_vfull = bar_kempty + 8 * C::NK;
   const uint32_t bar_vempty = bar_vfull + 8 * C::NV;
-  const uint32_t bar_sfull = bar_vempty + 8 * C::NV;
-  const uint32_t bar_pfull = bar_sfull + 16;
-  const uint32_t bar_odone = bar_pfull + 16;
-  const uint32_t bar_ofinal = bar_odone + 8;
+  const uint32_t bar_sfull = bar_vempty + 8 * C::NV;  // [2 buf]
+  const uint32_t bar_pfull = bar_sfull + 16;          // [2 buf][2 grp]
+  const uint32_t bar_pvdone = bar_pfull + 32;         // [2 buf]: the PV of a tile using S[buf] completed
+  const uint32_t bar_ofinal = bar_pvdone + 16;        // completes once per unit, after its last PV
   const uint32_t bar_list = bar_ofinal + 8;
-  const uint32_t bar_drain = bar_list + 8;
+  const uint32_t bar_drain = bar_list + 8;            // [2]: PV issuer, QK^T issuer
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint64_t limit = p.wait_limit_ns;
@@ -174,14 +182,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_vfull + 8 * s, 1);
       mbar_init(bar_vempty + 8 * s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar_sfull + 8 * b, 1);
-      mbar_init(bar_pfull + 8 * b, kSoftmaxThreads);
-    }
-    mbar_init(bar_odone, 1);
+    for (int b = 0; b < 2; ++b) mbar_init(bar_sfull + 8 * b, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(bar_pfull + 8 * i, kGroupWarps);  // one elected lane per warp
+    for (int b = 0; b < 2; ++b) mbar_init(bar_pvdone + 8 * b, 1);
     mbar_init(bar_ofinal, 1);
     mbar_init(bar_list, 1);
-    mbar_init(bar_drain, 1);
+    for (int i = 0; i < 2; ++i) mbar_init(bar_drain + 8 * i, 1);
     s_misc[MISC_ABORT] = 0;
     fence_mbar_init();
   }
@@ -278,69 +284,77 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     } else if (warp == 1) {
-      // ------------------------------------------------------------------ MMA issuer
+      // ------------------------------------------------------------------ PV issuer
+      if (lane == 0) {
+        int w = mbar_wait(bar_list, uphase, s_abort, limit);
+        if (w == WAIT_OK) {
+          const int T = s_misc[MISC_NK] + s_misc[MISC_NC];
+          constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+          // base descriptor; a K-step or stage offset is added to the start-address field
+          // (addresses stay below 256 KB, so the 14-bit field never carries)
+          const uint64_t vdesc0 = smem_desc_sw128(sb + C::OFF_V, C::CHUNK_BYTES, 1024);
+          for (int t = 0; t < T && w == WAIT_OK; ++t) {
+            const uint32_t g = tile_base + t;
+            const uint32_t b = g & 1u;
+            const int s = static_cast<int>(g % C::NV);
+            w = mbar_wait(bar_vfull + 8 * s, (g / C::NV) & 1u, s_abort, limit);
+            const uint64_t vd = vdesc0 + ((s * C::TILE_BYTES) >> 4);
+            // O_grp += P_grp V[64 grp .. 64 grp + 64), as soon as that group has written its P
+#pragma unroll
+            for (int grp = 0; grp < 2; ++grp) {
+              if (w == WAIT_OK) w = mbar_wait(bar_pfull + 8 * (2 * b + grp), (g >> 1) & 1u, s_abort, limit);
+              if (w == WAIT_OK) {
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  mma_bf16_ts(tmem + kColO + D * grp, tmem + kColS + 128 * b + 64 * grp + kk * 8,
+                              vd + (((4 * grp + kk) * 2048) >> 4), idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+                mma_issued = true;
+              }
+            }
+            if (w != WAIT_OK) break;
+            tc_commit(bar_vempty + 8 * s);
+            tc_commit(bar_pvdone + 8 * b);
+          }
+          if (w == WAIT_OK) tc_commit(bar_ofinal);
+        }
+        if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_MMA);
+      }
+    } else if (warp == kQkWarp) {
+      // ------------------------------------------------------------------ QK^T issuer
       if (lane == 0) {
         int w = mbar_wait(bar_list, uphase, s_abort, limit);
         if (w == WAIT_OK) w = mbar_wait(bar_q, uphase, s_abort, limit);
-        if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_MMA);
         if (w == WAIT_OK) {
           const int T = s_misc[MISC_NK] + s_misc[MISC_NC];
           constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
-          constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
-          const uint32_t q_addr = sb + C::OFF_Q;
-          bool ok = true;
-          for (int t = 0; t <= T && ok; ++t) {
-            if (t < T) {
-              const uint32_t g = tile_base + t;
-              const int s = static_cast<int>(g % C::NK);
-              const uint32_t b = g & 1u;
-              w = mbar_wait(bar_kfull + 8 * s, (g / C::NK) & 1u, s_abort, limit);
-              if (w != WAIT_OK) {
-                if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_MMA);
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              const uint32_t k_addr = sb + C::OFF_K + s * C::TILE_BYTES;
+          const uint64_t qdesc0 = smem_desc_sw128(sb + C::OFF_Q, 16, 1024);
+          const uint64_t kdesc0 = smem_desc_sw128(sb + C::OFF_K, 16, 1024);
+          for (int t = 0; t < T && w == WAIT_OK; ++t) {
+            const uint32_t g = tile_base + t;
+            const int s = static_cast<int>(g % C::NK);
+            const uint32_t b = g & 1u;
+            // S[b] holds the P of tile t-2 until that tile's PV has completed. pv_done[b] completes
+            // once per tile using S[b], and the PV of tile t cannot run before this QK^T, so the
+            // parity wait is exact. (Tiles of the previous unit completed before the unit ended.)
+            if (t >= 2) w = mbar_wait(bar_pvdone + 8 * b, ((g - 2u) >> 1) & 1u, s_abort, limit);
+            if (w == WAIT_OK) w = mbar_wait(bar_kfull + 8 * s, (g / C::NK) & 1u, s_abort, limit);
+            if (w != WAIT_OK) break;
+            tc_fence_after();
+            const uint64_t kd = kdesc0 + ((s * C::TILE_BYTES) >> 4);
 #pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
-                mma_bf16_ss(tmem + (b ? kColS1 : kColS0), smem_desc_sw128(q_addr + off, 16, 1024),
-                            smem_desc_sw128(k_addr + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-              }
-              mma_issued = true;
-              tc_commit(bar_sfull + 8 * b);
-              tc_commit(bar_kempty + 8 * s);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = ((kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32) >> 4;
+              mma_bf16_ss(tmem + kColS + 128 * b, qdesc0 + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
             }
-            if (t >= 1) {
-              // O += P V for the previous tile
-              const int tp = t - 1;
-              const uint32_t g = tile_base + tp;
-              const int s = static_cast<int>(g % C::NV);
-              const uint32_t b = g & 1u;
-              w = mbar_wait(bar_pfull + 8 * b, (g >> 1) & 1u, s_abort, limit);
-              if (w == WAIT_OK) w = mbar_wait(bar_vfull + 8 * s, (g / C::NV) & 1u, s_abort, limit);
-              if (w != WAIT_OK) {
-                if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_MMA);
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              const uint32_t v_addr = sb + C::OFF_V + s * C::TILE_BYTES;
-              const uint32_t p_col = tmem + (b ? kColP1 : kColP0);
-#pragma unroll
-              for (int kk = 0; kk < kRows / 16; ++kk) {
-                mma_bf16_ts(tmem + kColO, p_col + kk * 8, smem_desc_sw128(v_addr + kk * 2048, C::CHUNK_BYTES, 1024),
-                            idesc_pv, (tp > 0 || kk > 0) ? 1u : 0u);
-              }
-              tc_commit(bar_vempty + 8 * s);
-              tc_commit(bar_odone);
-            }
+            mma_issued = true;
+            tc_commit(bar_sfull + 8 * b);
+            tc_commit(bar_kempty + 8 * s);
           }
-          if (ok) tc_commit(bar_ofinal);
         }
+        if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_MMA);
       }
-    } else if (warp >= kSoftmaxWarp0) {
+    } else {
       // ------------------------------------------------------------------ router + softmax + epilogue
       const int st = tid - kSoftmaxWarp0 * 32;  // 0..255
       const int grp = st >> 7;                  // column half: warps 2..5 -> 0, warps 6..9 -> 1
@@ -471,76 +485,77 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 
       // (2)+(3) online softmax over kept tiles, then pooled tiles; this thread: row `row`,
-      // score columns [64 grp, 64 grp + 64)
+      // score columns [64 grp, 64 grp + 64), its own running max, sum and accumulator O_grp
       const int nk = s_misc[MISC_NK];
       const int T = alive ? nk + s_misc[MISC_NC] : 0;
       const float sl2 = p.sl2;
+      const uint32_t o_col = tmem + lane_base + kColO + D * grp;
       float m_run = -INFINITY, l_run = 0.f;
       bool bad = false;  // a wait of this warp failed inside the tile loop
       for (int t = 0; t < T; ++t) {
         const uint32_t g = tile_base + t;
         const uint32_t b = g & 1u;
+        const uint32_t s_col = tmem + lane_base + kColS + 128 * b + 64 * grp;
         w = mbar_wait(bar_sfull + 8 * b, (g >> 1) & 1u, s_abort, limit);
         if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_SOFTMAX);
-        const bool ok = __all_sync(0xffffffffu, w == WAIT_OK) && !bad;
+        if (!__all_sync(0xffffffffu, w == WAIT_OK)) {
+          bad = true;
+          break;
+        }
+        tc_fence_after();
         float s[64];
-        float mx = -INFINITY;
         const bool exact = t < nk;
         const int j = exact ? static_cast<int>(s_klist[t]) : 0;
         const bool full = exact && (j != nkb - 1 || p.last_n == kRows);
-        if (ok) {
-          tc_fence_after();
+        {
           uint32_t raw[64];
-          tmem_ld_x64(tmem + lane_base + (b ? kColS1 : kColS0) + grp * 64, raw);
+          tmem_ld_x64(s_col, raw);
 #pragma unroll
           for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(raw[c]);
-          if (full) {
-            mx = max64(s) * sl2;  // sl2 > 0: the max of the scaled scores
+        }
+        float mx;
+        if (full) {
+          mx = max64(s) * sl2;  // sl2 > 0: the max of the scaled scores
+        } else {
+          if (exact) {
+            const int valid = p.last_n - grp * 64;  // valid columns in this half (may be <= 0)
+#pragma unroll
+            for (int c = 0; c < 64; ++c) s[c] = (c < valid) ? s[c] * sl2 : -INFINITY;
           } else {
-            if (exact) {
-              const int valid = p.last_n - grp * 64;  // valid columns in this half
+            const int cc = s_clist[t - nk];
+            const int valid = min(kRows, nkb - cc * kRows) - grp * 64;
+            const int nwords = (nkb + 31) / 32;
+            const uint32_t kw0 = (cc * 4 + grp * 2 < nwords) ? s_bits[cc * 4 + grp * 2] : 0u;
+            const uint32_t kw1 = (cc * 4 + grp * 2 + 1 < nwords) ? s_bits[cc * 4 + grp * 2 + 1] : 0u;
+            const int last_col = nkb - 1 - cc * kRows - grp * 64;  // column of the ragged last block, if here
 #pragma unroll
-              for (int c = 0; c < 64; ++c) s[c] = (c < valid) ? s[c] * sl2 : -INFINITY;
-            } else {
-              const int cc = s_clist[t - nk];
-              const int valid = min(kRows, nkb - cc * kRows) - grp * 64;
-              const int nwords = (nkb + 31) / 32;
-              const uint32_t kw0 = (cc * 4 + grp * 2 < nwords) ? s_bits[cc * 4 + grp * 2] : 0u;
-              const uint32_t kw1 = (cc * 4 + grp * 2 + 1 < nwords) ? s_bits[cc * 4 + grp * 2 + 1] : 0u;
-              const int last_col = nkb - 1 - cc * kRows - grp * 64;  // column of the ragged last block, if here
-#pragma unroll
-              for (int c = 0; c < 64; ++c) {
-                const uint32_t kw = c < 32 ? kw0 : kw1;
-                const bool skipped = c < valid && !((kw >> (c & 31)) & 1u);
-                const float off = (c == last_col) ? p.log2_last_n : 7.0f;  // log2(n_j)
-                s[c] = skipped ? fmaf(s[c], sl2, off) : -INFINITY;
-              }
+            for (int c = 0; c < 64; ++c) {
+              const uint32_t kw = c < 32 ? kw0 : kw1;
+              const bool skipped = c < valid && !((kw >> (c & 31)) & 1u);
+              const float off = (c == last_col) ? p.log2_last_n : 7.0f;  // log2(n_j)
+              s[c] = skipped ? fmaf(s[c], sl2, off) : -INFINITY;
             }
-            mx = max64(s);
           }
+          mx = max64(s);
         }
-        // exchange the half-row maxima; the vote makes every softmax thread leave together
-        s_xmax[(b * 2 + grp) * kRows + row] = mx;
-        if (named_barrier_or(kBarSoftmax, kSoftmaxThreads, !ok)) {
-          alive = false;
-          break;
-        }
-        const float mt = fmaxf(s_xmax[(b * 2 + 0) * kRows + row], s_xmax[(b * 2 + 1) * kRows + row]);
+        // lazy rescale; a half row whose columns have all been masked so far keeps m = -inf and
+        // P = 0, and the first finite max rescales its (zero) accumulator by 0
         float m_new = m_run, alpha = 1.f;
         bool need = false;
         if (t == 0) {
-          m_new = mt;
-        } else if (mt > m_run + kRescaleThreshold) {
+          m_new = mx;
+        } else if (mx > m_run + kRescaleThreshold) {
           need = true;
-          m_new = mt;
-          alpha = ex2_approx(m_run - mt);
+          m_new = mx;
+          alpha = ex2_approx(m_run - mx);
         }
         m_run = m_new;
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
         uint32_t pk[32];
         float acc[4] = {0.f, 0.f, 0.f, 0.f};  // row sum of the bf16-rounded weights, 4 chains
         if (full) {
           const float2 scale2 = make_float2(sl2, sl2);
-          const float2 negm2 = make_float2(-m_new, -m_new);
+          const float2 negm2 = make_float2(-m_use, -m_use);
 #pragma unroll
           for (int c2 = 0; c2 < 32; ++c2) {
             const float2 x2 = __ffma2_rn(make_float2(s[2 * c2], s[2 * c2 + 1]), scale2, negm2);
@@ -556,40 +571,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
 #pragma unroll
           for (int c2 = 0; c2 < 32; ++c2) {
-            const float e0 = ex2_approx(s[2 * c2] - m_new);
-            const float e1 = ex2_approx(s[2 * c2 + 1] - m_new);
+            const float e0 = ex2_approx(s[2 * c2] - m_use);
+            const float e1 = ex2_approx(s[2 * c2 + 1] - m_use);
             pk[c2] = pack_bf16x2(e0, e1);
             acc[c2 & 3] = add_bf16x2(acc[c2 & 3], pk[c2]);
           }
         }
         // the row sum takes the same bf16-rounded weights the PV MMA uses
         l_run = fmaf(l_run, alpha, (acc[0] + acc[1]) + (acc[2] + acc[3]));
-        tmem_st_x32(tmem + lane_base + (b ? kColP1 : kColP0) + grp * 32, pk);
+        // P over the first 32 of this group's S columns, which are already in registers
+        tmem_st_x32(s_col, pk);
         if (__any_sync(0xffffffffu, need)) {
-          // rescale this group's half of O after the previous tile's PV has landed
-          w = mbar_wait(bar_odone, (g - 1u) & 1u, s_abort, limit);
+          // rescale O_grp once the previous tile's PV has landed. pv_done[buf] completes once per
+          // tile using that buffer; the PV three tiles back completed before the one two tiles back
+          // (same accumulators, same issuing thread), which completed before this tile's QK^T was
+          // issued, and the PV of tile t+1 needs this group's next P, so the parity wait is exact.
+          w = mbar_wait(bar_pvdone + 8 * ((g - 1u) & 1u), ((g - 1u) >> 1) & 1u, s_abort, limit);
           if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_SOFTMAX);
           if (__all_sync(0xffffffffu, w == WAIT_OK)) {
             tc_fence_after();
 #pragma unroll 1
-            for (int ch = 0; ch < D / 64; ++ch) {
+            for (int ch = 0; ch < D / 32; ++ch) {
               uint32_t o[32];
-              const uint32_t oc = tmem + lane_base + kColO + grp * (D / 2) + ch * 32;
-              tmem_ld_x32(oc, o);
+              tmem_ld_x32(o_col + ch * 32, o);
 #pragma unroll
               for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-              tmem_st_x32(oc, o);
+              tmem_st_x32(o_col + ch * 32, o);
             }
           } else {
-            bad = true;  // leave at the next vote; P is still published so nothing else blocks
+            bad = true;  // P is still published below, so the MMA issuer is not left waiting
           }
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar_pfull + 8 * b);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_pfull + 8 * (2 * b + grp));
+        if (bad) break;
       }
 
-      // (4) epilogue: combine the two half-row sums, O / l -> bf16, each group stores its columns
+      // (4) epilogue: merge the two groups' partial results, O / l -> bf16; group g stores
+      // output columns [g D/2, (g+1) D/2)
       {
         bool ok = alive && !bad && T > 0;
         if (ok) {
@@ -597,23 +618,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_SOFTMAX);
           ok = __all_sync(0xffffffffu, w == WAIT_OK);
         }
-        // every softmax thread reaches this barrier: the tile loop is left by all of them together
-        s_lsum[grp * kRows + row] = l_run;
+        // every softmax thread reaches this barrier, whether or not its tile loop ended early
+        s_ml[grp * kRows + row] = make_float2(m_run, l_run);
         const bool any_bad = named_barrier_or(kBarSoftmax, kSoftmaxThreads, !ok);
         if (!any_bad) {
           tc_fence_after();
-          const float inv = 1.f / (s_lsum[row] + s_lsum[kRows + row]);
+          const float2 ml0 = s_ml[row], ml1 = s_ml[kRows + row];
+          const float m = fmaxf(ml0.x, ml1.x);  // finite: every row sees at least one valid column
+          const float a0 = ex2_approx(ml0.x - m), a1 = ex2_approx(ml1.x - m);  // 2^-inf = 0
+          const float inv = 1.f / fmaf(ml0.y, a0, ml1.y * a1);
+          const float c0 = a0 * inv, c1 = a1 * inv;
           const bool store = row < m_i;
           __nv_bfloat16* dst = p.O + (static_cast<size_t>(bh) * p.L + static_cast<size_t>(qb) * kRows + row) * D +
                                grp * (D / 2);
+          const uint32_t o0 = tmem + lane_base + kColO + grp * (D / 2);
 #pragma unroll
           for (int ch = 0; ch < D / 64; ++ch) {
-            uint32_t o[32];
-            tmem_ld_x32(tmem + lane_base + kColO + grp * (D / 2) + ch * 32, o);
+            uint32_t x0[32], x1[32];
+            tmem_ld_x32(o0 + ch * 32, x0);
+            tmem_ld_x32(o0 + D + ch * 32, x1);
             uint32_t pkd[16];
 #pragma unroll
             for (int c = 0; c < 16; ++c)
-              pkd[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv, __uint_as_float(o[2 * c + 1]) * inv);
+              pkd[c] = pack_bf16x2(fmaf(__uint_as_float(x0[2 * c]), c0, __uint_as_float(x1[2 * c]) * c1),
+                                   fmaf(__uint_as_float(x0[2 * c + 1]), c0, __uint_as_float(x1[2 * c + 1]) * c1));
             if (store) {
               uint4* d4 = reinterpret_cast<uint4*>(dst + ch * 32);
 #pragma unroll
@@ -632,9 +660,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ---- drain: no copy or MMA may still be in flight when TMEM and shared memory are released
-  if (warp == 1 && lane == 0 && mma_issued) {
-    tc_commit(bar_drain);
-    mbar_wait(bar_drain, 0, nullptr, limit);
+  if ((warp == 1 || warp == kQkWarp) && lane == 0 && mma_issued) {
+    const uint32_t bd = bar_drain + (warp == 1 ? 0 : 8);
+    tc_commit(bd);
+    mbar_wait(bd, 0, nullptr, limit);
   }
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < C::NK; ++s)
