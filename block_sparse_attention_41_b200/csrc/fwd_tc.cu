@@ -14,11 +14,12 @@
 //                 MMA/softmax pipeline and the same running max, sum and accumulator.
 //   4. epilogue : O / l -> bf16 -> global.
 //
-// Roles (352 threads): warp 0 = TMA producer, warp 1 = PV issuer (also owns TMEM), warps 2..5
-// and 6..9 = two softmax groups, warp 10 = QK^T issuer. A tcgen05.mma blocks its issuing thread
-// for about as long as the tensor pipe takes to run it, so the two products are issued from two
-// threads: waiting for one tile's PV to finish (before its S buffer is refilled) never delays the
-// PV of the next tile. A warp may only touch TMEM lanes 32*(warp%4) .. +31, and any four
+// Roles (384 threads): warp 0 = TMA producer, warps 1 and 11 = PV issuers of softmax groups 0
+// and 1 (warp 1 also owns TMEM), warps 2..5 and 6..9 = the two softmax groups, warp 10 = QK^T
+// issuer. A tcgen05.mma blocks its issuing thread for about as long as the tensor pipe takes to
+// run it, so the products are issued from three threads: a group's PV starts as soon as that
+// group's P is written, and waiting for one tile's PV to finish (before its S buffer is refilled)
+// never delays the PV of the next tile. A warp may only touch TMEM lanes 32*(warp%4) .. +31, and any four
 // consecutive warps cover all four quarters, so thread (g, r) of softmax group g owns query
 // row r (TMEM lane r) and score columns [64g, 64g+64) of every tile.
 //
@@ -34,10 +35,9 @@
 // while the softmax works on tile t+1. K tiles go round a 3-deep ring (d = 128) and are released
 // as soon as their QK^T completes; V tiles go round a 2-deep ring and are released after PV.
 //
-// Exponentials: ex2.approx on the MUFU unit, except one column pair in four of every full
-// exact tile. Those use 2^x = 2^floor(x) * p(x - floor(x)), where p is a cubic minimax fit of 2^f
-// on [0, 1) (max relative error 8.6e-5, far below the bf16 rounding of P), evaluated with
-// packed f32x2 FMAs. That moves part of the exponential work from MUFU to the FMA pipe.
+// Exponentials: ex2.approx on the MUFU unit. An optional path (kPolyEvery) computes some of them
+// on the FMA pipe as 2^x = 2^floor(x) * p(x - floor(x)), where p is a cubic minimax fit of 2^f on
+// [0, 1) (max relative error 8.6e-5, far below the bf16 rounding of P).
 //
 // Every mbarrier wait is bounded (sol::mbar_wait). On expiry the CTA records SOL_ETIMEOUT in the
 // workspace, the other roles stop at their next wait, in-flight copies and MMAs are drained, and
@@ -52,9 +52,10 @@ namespace sol {
 
 namespace {
 
-constexpr int kThreads = 352;
+constexpr int kThreads = 384;
 constexpr int kSoftmaxWarp0 = 2;
 constexpr int kQkWarp = 10;
+constexpr int kPv1Warp = 11;  // PV issuer of softmax group 1 (group 0's is warp 1)
 constexpr int kSoftmaxThreads = 256;
 constexpr int kGroupWarps = 4;  // warps per softmax group
 constexpr int kRows = 128;      // B_q = B_k
@@ -66,6 +67,10 @@ constexpr uint32_t kBarSoftmax = 1;       // named barrier of the 256 softmax th
 
 // cubic minimax fit of 2^f on [0, 1] with p(0) = 1 (relative error <= 8.6e-5)
 constexpr float kExpC1 = 0.69511664f, kExpC2 = 0.22764498f, kExpC3 = 0.07706724f;
+// Column pairs of a full exact tile whose exponentials take the polynomial: pair c with
+// c % kPolyEvery == kPolyEvery - 1; 0 = none. Measured on B200 with this pipeline, moving work off
+// MUFU costs more issue slots than it saves, so it is off.
+constexpr int kPolyEvery = 0;
 
 template <int D>
 struct TcCfg {
@@ -87,8 +92,8 @@ struct TcCfg {
   static constexpr int OFF_MISC = OFF_RED + 32;                           // int[8]
   static constexpr int OFF_BAR = OFF_MISC + 32;                           // mbarriers
   // q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2], p_full[2 buf][2 grp],
-  // pv_done[2 buf], o_final, list_ready, drain[2 issuers]
-  static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 2 + 4 + 2 + 1 + 1 + 2;
+  // pv_done[2 buf], o_final, list_ready, drain[3 issuers]
+  static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 2 + 4 + 2 + 1 + 1 + 3;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;  // + slack to align the base to 1024 B
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -167,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_pvdone = bar_pfull + 32;         // [2 buf]: the PV of a tile using S[buf] completed
   const uint32_t bar_ofinal = bar_pvdone + 16;        // completes once per unit, after its last PV
   const uint32_t bar_list = bar_ofinal + 8;
-  const uint32_t bar_drain = bar_list + 8;            // [2]: PV issuer, QK^T issuer
+  const uint32_t bar_drain = bar_list + 8;            // [3]: PV issuers of groups 0 and 1, QK^T issuer
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint64_t limit = p.wait_limit_ns;
@@ -180,14 +185,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < C::NV; ++s) {
       mbar_init(bar_vfull + 8 * s, 1);
-      mbar_init(bar_vempty + 8 * s, 1);
+      mbar_init(bar_vempty + 8 * s, 2);  // both PV issuers commit
     }
     for (int b = 0; b < 2; ++b) mbar_init(bar_sfull + 8 * b, 1);
     for (int i = 0; i < 4; ++i) mbar_init(bar_pfull + 8 * i, kGroupWarps);  // one elected lane per warp
-    for (int b = 0; b < 2; ++b) mbar_init(bar_pvdone + 8 * b, 1);
-    mbar_init(bar_ofinal, 1);
+    for (int b = 0; b < 2; ++b) mbar_init(bar_pvdone + 8 * b, 2);  // both PV issuers commit
+    mbar_init(bar_ofinal, 2);
     mbar_init(bar_list, 1);
-    for (int i = 0; i < 2; ++i) mbar_init(bar_drain + 8 * i, 1);
+    for (int i = 0; i < 3; ++i) mbar_init(bar_drain + 8 * i, 1);
     s_misc[MISC_ABORT] = 0;
     fence_mbar_init();
   }
@@ -283,8 +288,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-    } else if (warp == 1) {
-      // ------------------------------------------------------------------ PV issuer
+    } else if (warp == 1 || warp == kPv1Warp) {
+      // ------------------------------------------------------------------ PV issuers
+      // O_grp += P_grp V[64 grp .. 64 grp + 64): one thread per softmax group
+      const int grp = warp == 1 ? 0 : 1;
       if (lane == 0) {
         int w = mbar_wait(bar_list, uphase, s_abort, limit);
         if (w == WAIT_OK) {
@@ -292,27 +299,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
           // base descriptor; a K-step or stage offset is added to the start-address field
           // (addresses stay below 256 KB, so the 14-bit field never carries)
-          const uint64_t vdesc0 = smem_desc_sw128(sb + C::OFF_V, C::CHUNK_BYTES, 1024);
+          const uint64_t vdesc0 = smem_desc_sw128(sb + C::OFF_V, C::CHUNK_BYTES, 1024) + ((4 * grp * 2048) >> 4);
+          const uint32_t o_acc = tmem + kColO + D * grp;
           for (int t = 0; t < T && w == WAIT_OK; ++t) {
             const uint32_t g = tile_base + t;
             const uint32_t b = g & 1u;
             const int s = static_cast<int>(g % C::NV);
-            w = mbar_wait(bar_vfull + 8 * s, (g / C::NV) & 1u, s_abort, limit);
-            const uint64_t vd = vdesc0 + ((s * C::TILE_BYTES) >> 4);
-            // O_grp += P_grp V[64 grp .. 64 grp + 64), as soon as that group has written its P
-#pragma unroll
-            for (int grp = 0; grp < 2; ++grp) {
-              if (w == WAIT_OK) w = mbar_wait(bar_pfull + 8 * (2 * b + grp), (g >> 1) & 1u, s_abort, limit);
-              if (w == WAIT_OK) {
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                  mma_bf16_ts(tmem + kColO + D * grp, tmem + kColS + 128 * b + 64 * grp + kk * 8,
-                              vd + (((4 * grp + kk) * 2048) >> 4), idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
-                mma_issued = true;
-              }
-            }
+            w = mbar_wait(bar_pfull + 8 * (2 * b + grp), (g >> 1) & 1u, s_abort, limit);
+            if (w == WAIT_OK) w = mbar_wait(bar_vfull + 8 * s, (g / C::NV) & 1u, s_abort, limit);
             if (w != WAIT_OK) break;
+            tc_fence_after();
+            const uint64_t vd = vdesc0 + ((s * C::TILE_BYTES) >> 4);
+            const uint32_t p_col = tmem + kColS + 128 * b + 64 * grp;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ts(o_acc, p_col + kk * 8, vd + ((kk * 2048) >> 4), idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+            mma_issued = true;
             tc_commit(bar_vempty + 8 * s);
             tc_commit(bar_pvdone + 8 * b);
           }
@@ -560,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c2 = 0; c2 < 32; ++c2) {
             const float2 x2 = __ffma2_rn(make_float2(s[2 * c2], s[2 * c2 + 1]), scale2, negm2);
             float2 e2;
-            if ((c2 & 3) == 3) {
+            if (kPolyEvery > 0 && (c2 % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
               e2 = exp2_poly2(make_float2(fmaxf(x2.x, -126.f), fmaxf(x2.y, -126.f)));
             } else {
               e2 = make_float2(ex2_approx(x2.x), ex2_approx(x2.y));
@@ -660,8 +662,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ---- drain: no copy or MMA may still be in flight when TMEM and shared memory are released
-  if ((warp == 1 || warp == kQkWarp) && lane == 0 && mma_issued) {
-    const uint32_t bd = bar_drain + (warp == 1 ? 0 : 8);
+  if ((warp == 1 || warp == kPv1Warp || warp == kQkWarp) && lane == 0 && mma_issued) {
+    const uint32_t bd = bar_drain + (warp == 1 ? 0 : (warp == kPv1Warp ? 8 : 16));
     tc_commit(bd);
     mbar_wait(bd, 0, nullptr, limit);
   }
