@@ -86,7 +86,7 @@ struct TcCfg {
   static constexpr int OFF_KLIST = OFF_SBAR + kMaxKeyBlocks * 4;          // u16[kMaxKeyBlocks]
   static constexpr int OFF_BITS = OFF_KLIST + kMaxKeyBlocks * 2;          // u32[kMaxKeyBlocks/32]
   static constexpr int OFF_CLIST = OFF_BITS + kMaxKeyBlocks / 8;          // u16[kMaxKeyBlocks/128]
-  static constexpr int OFF_QBAR = OFF_CLIST + (kMaxKeyBlocks / 128) * 2;  // float[D] + float[256] partials
+  static constexpr int OFF_QBAR = OFF_CLIST + (kMaxKeyBlocks / 128) * 2;  // float[D] + int[256] word prefixes
   static constexpr int OFF_ML = OFF_QBAR + (D + kSoftmaxThreads) * 4;     // float2[2 grp][128 rows]
   static constexpr int OFF_RED = OFF_ML + 2 * kRows * 8;                  // float[8]
   static constexpr int OFF_MISC = OFF_RED + 32;                           // int[8]
@@ -97,6 +97,8 @@ struct TcCfg {
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;  // + slack to align the base to 1024 B
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(kMaxKeyBlocks / 32 <= kSoftmaxThreads, "word prefixes fit after q_bar");
+  static_assert((kSoftmaxThreads / (D / 8)) * D <= kMaxKeyBlocks, "q_bar partial sums fit in the proxy-score buffer");
   static_assert(kColO + 2 * D <= kTmemCols, "TMEM budget");
 };
 
@@ -369,44 +371,59 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       int w = mbar_wait(bar_q, uphase, s_abort, limit);
       if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_ROUTER);
-      bool alive = !named_barrier_or(kBarSoftmax, kSoftmaxThreads, w != WAIT_OK);  // same in all 256
+      const bool alive = !named_barrier_or(kBarSoftmax, kSoftmaxThreads, w != WAIT_OK);  // same in all 256
 
-      // (1a) q_bar = mean of the valid query rows, read from the swizzled Q tile
+      // (1a) q_bar = mean of the valid query rows, read from the swizzled Q tile. Thread st sums one
+      // 16-byte chunk (8 columns) over a strided set of rows; the partial sums meet in shared memory
+      // (the proxy-score buffer, not yet in use).
       {
-        constexpr int TPC = kSoftmaxThreads / D;  // threads per column: 2 (D=128) or 4 (D=64)
-        const int c = st % D, part = st / D;
-        const uint8_t* qt = smem + C::OFF_Q + (c >> 6) * C::CHUNK_BYTES;
-        const int cw = c & 63;
-        float acc = 0.f;
+        constexpr int CH = D / 8;                  // 16-byte chunks per row
+        constexpr int RG = kSoftmaxThreads / CH;   // row groups: 16 (D=128) or 32 (D=64)
+        const int c8 = st % CH, rg = st / CH;
+        const uint8_t* qt = smem + C::OFF_Q + (c8 >> 3) * C::CHUNK_BYTES;
+        const int jc = c8 & 7;
+        float a[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) a[k] = 0.f;
         if (alive) {
-          for (int r = part; r < m_i; r += TPC) {
-            const uint32_t off = r * 128 + ((((cw >> 3) ^ (r & 7))) << 4) + ((cw & 7) << 1);
-            acc += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(qt + off));
+#pragma unroll 2
+          for (int r = rg; r < m_i; r += RG) {
+            const uint4 v = *reinterpret_cast<const uint4*>(qt + r * 128 + ((jc ^ (r & 7)) << 4));
+            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              a[2 * k] += __uint_as_float(wv[k] << 16);
+              a[2 * k + 1] += __uint_as_float(wv[k] & 0xffff0000u);
+            }
           }
         }
-        s_qbar[D + st] = acc;
+        float* part = s_sbar;  // [RG][D]
+#pragma unroll
+        for (int k = 0; k < 8; ++k) part[rg * D + c8 * 8 + k] = a[k];
         named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
         if (st < D) {
-          float s = 0.f;
-#pragma unroll
-          for (int k = 0; k < TPC; ++k) s += s_qbar[D + st + k * D];
-          s_qbar[st] = s / static_cast<float>(m_i);
+          float q = 0.f;
+#pragma unroll 8
+          for (int k = 0; k < RG; ++k) q += part[k * D + st];
+          s_qbar[st] = q / static_cast<float>(m_i);
         }
         named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
       }
 
-      // (1b) proxy scores s_bar_j (shared memory only) and their max; 8 warps, 4 rows in flight each
+      // (1b) proxy scores s_bar_j (shared memory only) and their max; 8 warps, 16 rows in flight
+      // each (the pooled keys come from L2, so the loop is bound by how many loads are in flight)
       {
         constexpr int DPL = D / 32;
+        constexpr int U = 16;
         float qv[DPL];
 #pragma unroll
         for (int k = 0; k < DPL; ++k) qv[k] = s_qbar[lane * DPL + k];
         const float* kb = p.kbar + static_cast<size_t>(bh) * nkb * D + lane * DPL;
         float wmax = -INFINITY;
-        for (int j0 = sw; j0 < nkb; j0 += 32) {
-          float dot[4];
+        for (int j0 = sw; j0 < nkb; j0 += 8 * U) {
+          float dot[U];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int u = 0; u < U; ++u) {
             const int j = j0 + 8 * u;
             dot[u] = 0.f;
             if (j < nkb) {
@@ -423,15 +440,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) dot[u] += __shfl_xor_sync(0xffffffffu, dot[u], o);
+            for (int u = 0; u < U; ++u) dot[u] += __shfl_xor_sync(0xffffffffu, dot[u], o);
           }
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int u = 0; u < U; ++u) {
             const int j = j0 + 8 * u;
             if (j < nkb) {
-              const float s = dot[u] * p.inv_sqrt_d;
-              if (lane == 0) s_sbar[j] = s;
-              wmax = fmaxf(wmax, s);
+              const float sc = dot[u] * p.inv_sqrt_d;
+              if (lane == 0) s_sbar[j] = sc;
+              wmax = fmaxf(wmax, sc);
             }
           }
         }
@@ -439,43 +456,64 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
       }
 
-      // (1c) keep bits, kept list, pooled-tile list (softmax warp 0)
-      if (sw == 0) {
+      // (1c) keep bits (each warp ballots whole words), their prefix counts (warp 0), then the kept
+      // list and the pooled-tile list
+      {
         float M = s_red[0];
 #pragma unroll
         for (int k = 1; k < 8; ++k) M = fmaxf(M, s_red[k]);
         const float thr = M - p.tau[bh % p.H];
-        int nk = 0;
-        for (int base = 0; base < nkb; base += 32) {
-          const int j = base + lane;
+        const int nwords = (nkb + 31) / 32;
+        for (int i = sw; i < nwords; i += 8) {
+          const int j = 32 * i + lane;
           const bool k = j < nkb && (s_sbar[j] >= thr || j < p.n_force);
           const uint32_t m = __ballot_sync(0xffffffffu, k);
-          if (lane == 0) s_bits[base >> 5] = m;
-          if (k) s_klist[nk + __popc(m & ((1u << lane) - 1u))] = static_cast<uint16_t>(j);
-          nk += __popc(m);
+          if (lane == 0) s_bits[i] = m;
         }
-        __syncwarp();
-        const int nchunks = (nkb + kRows - 1) / kRows;
-        int nc = 0;
-        for (int cb = 0; cb < nchunks; cb += 32) {
-          const int cc = cb + lane;
-          bool has_skip = false;
-          if (cc < nchunks) {
-            const int valid = min(kRows, nkb - cc * kRows);
-            int kept = 0;
+        named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
+        int* s_pref = reinterpret_cast<int*>(s_qbar + D);  // [kMaxKeyBlocks / 32]: kept blocks before word i
+        if (sw == 0) {
+          int run = 0;
+          for (int i0 = 0; i0 < nwords; i0 += 32) {
+            const int i = i0 + lane;
+            const int c = i < nwords ? __popc(s_bits[i]) : 0;
+            int x = c;  // inclusive warp scan
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              if (cc * 4 + q < (nkb + 31) / 32) kept += __popc(s_bits[cc * 4 + q]);
-            has_skip = kept < valid;
+            for (int o = 1; o < 32; o <<= 1) {
+              const int y = __shfl_up_sync(0xffffffffu, x, o);
+              if (lane >= o) x += y;
+            }
+            if (i < nwords) s_pref[i] = run + x - c;
+            run += __shfl_sync(0xffffffffu, x, 31);
           }
-          const uint32_t m = __ballot_sync(0xffffffffu, has_skip);
-          if (has_skip) s_clist[nc + __popc(m & ((1u << lane) - 1u))] = static_cast<uint16_t>(cc);
-          nc += __popc(m);
+          const int nk = run;
+          const int nchunks = (nkb + kRows - 1) / kRows;
+          int nc = 0;
+          for (int cb = 0; cb < nchunks; cb += 32) {
+            const int cc = cb + lane;
+            bool has_skip = false;
+            if (cc < nchunks) {
+              const int valid = min(kRows, nkb - cc * kRows);
+              int kept = 0;
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                if (cc * 4 + q < nwords) kept += __popc(s_bits[cc * 4 + q]);
+              has_skip = kept < valid;
+            }
+            const uint32_t m = __ballot_sync(0xffffffffu, has_skip);
+            if (has_skip) s_clist[nc + __popc(m & ((1u << lane) - 1u))] = static_cast<uint16_t>(cc);
+            nc += __popc(m);
+          }
+          if (lane == 0) {
+            s_misc[MISC_NK] = alive ? nk : 0;
+            s_misc[MISC_NC] = alive ? nc : 0;
+            atomicAdd(&p.ws[WS_COUNTS + bh], static_cast<uint32_t>(nk));
+          }
         }
-        if (lane == 0) {
-          s_misc[MISC_NK] = alive ? nk : 0;
-          s_misc[MISC_NC] = alive ? nc : 0;
-          atomicAdd(&p.ws[WS_COUNTS + bh], static_cast<uint32_t>(nk));
+        named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
+        for (int i = sw; i < nwords; i += 8) {
+          const uint32_t m = s_bits[i];
+          if ((m >> lane) & 1u) s_klist[s_pref[i] + __popc(m & ((1u << lane) - 1u))] = static_cast<uint16_t>(32 * i + lane);
         }
       }
       named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
