@@ -103,7 +103,8 @@ struct TcCfg {
 };
 
 struct TcParams {
-  const float* kbar;  // fp32 [BH, nkb, D] routing proxy
+  const float* kbar;          // fp32 [BH, nkb, D] routing proxy
+  const uint32_t* bits;       // [BH * nqb, ceil(nkb / 32)] keep bits from the routing pass, or null
   __nv_bfloat16* O;
   uint8_t* kept_mask;
   float* density;
@@ -369,108 +370,119 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int m_i = min(kRows, p.L - qb * kRows);
       const int nkb = p.nkb;
 
-      int w = mbar_wait(bar_q, uphase, s_abort, limit);
-      if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_ROUTER);
-      const bool alive = !named_barrier_or(kBarSoftmax, kSoftmaxThreads, w != WAIT_OK);  // same in all 256
+      const int nwords = (nkb + 31) / 32;
+      int w = WAIT_OK;
+      bool alive = true;  // same in all 256
+      if (p.bits != nullptr) {
+        // (1) the unit was routed by the routing pass: its keep bits
+        const uint32_t* ub = p.bits + static_cast<size_t>(unit) * nwords;
+        for (int i = st; i < nwords; i += kSoftmaxThreads) s_bits[i] = __ldg(ub + i);
+      } else {
+        w = mbar_wait(bar_q, uphase, s_abort, limit);
+        if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_ROUTER);
+        alive = !named_barrier_or(kBarSoftmax, kSoftmaxThreads, w != WAIT_OK);
 
-      // (1a) q_bar = mean of the valid query rows, read from the swizzled Q tile. Thread st sums one
-      // 16-byte chunk (8 columns) over a strided set of rows; the partial sums meet in shared memory
-      // (the proxy-score buffer, not yet in use).
-      {
-        constexpr int CH = D / 8;                  // 16-byte chunks per row
-        constexpr int RG = kSoftmaxThreads / CH;   // row groups: 16 (D=128) or 32 (D=64)
-        const int c8 = st % CH, rg = st / CH;
-        const uint8_t* qt = smem + C::OFF_Q + (c8 >> 3) * C::CHUNK_BYTES;
-        const int jc = c8 & 7;
-        float a[8];
+        // (1a) q_bar = mean of the valid query rows, read from the swizzled Q tile. Thread st sums one
+        // 16-byte chunk (8 columns) over a strided set of rows; the partial sums meet in shared memory
+        // (the proxy-score buffer, not yet in use).
+        {
+          constexpr int CH = D / 8;                  // 16-byte chunks per row
+          constexpr int RG = kSoftmaxThreads / CH;   // row groups: 16 (D=128) or 32 (D=64)
+          const int c8 = st % CH, rg = st / CH;
+          const uint8_t* qt = smem + C::OFF_Q + (c8 >> 3) * C::CHUNK_BYTES;
+          const int jc = c8 & 7;
+          float a[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) a[k] = 0.f;
-        if (alive) {
+          for (int k = 0; k < 8; ++k) a[k] = 0.f;
+          if (alive) {
 #pragma unroll 2
-          for (int r = rg; r < m_i; r += RG) {
-            const uint4 v = *reinterpret_cast<const uint4*>(qt + r * 128 + ((jc ^ (r & 7)) << 4));
-            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+            for (int r = rg; r < m_i; r += RG) {
+              const uint4 v = *reinterpret_cast<const uint4*>(qt + r * 128 + ((jc ^ (r & 7)) << 4));
+              const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              a[2 * k] += __uint_as_float(wv[k] << 16);
-              a[2 * k + 1] += __uint_as_float(wv[k] & 0xffff0000u);
-            }
-          }
-        }
-        float* part = s_sbar;  // [RG][D]
-#pragma unroll
-        for (int k = 0; k < 8; ++k) part[rg * D + c8 * 8 + k] = a[k];
-        named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
-        if (st < D) {
-          float q = 0.f;
-#pragma unroll 8
-          for (int k = 0; k < RG; ++k) q += part[k * D + st];
-          s_qbar[st] = q / static_cast<float>(m_i);
-        }
-        named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
-      }
-
-      // (1b) proxy scores s_bar_j (shared memory only) and their max; 8 warps, 16 rows in flight
-      // each (the pooled keys come from L2, so the loop is bound by how many loads are in flight)
-      {
-        constexpr int DPL = D / 32;
-        constexpr int U = 16;
-        float qv[DPL];
-#pragma unroll
-        for (int k = 0; k < DPL; ++k) qv[k] = s_qbar[lane * DPL + k];
-        const float* kb = p.kbar + static_cast<size_t>(bh) * nkb * D + lane * DPL;
-        float wmax = -INFINITY;
-        for (int j0 = sw; j0 < nkb; j0 += 8 * U) {
-          float dot[U];
-#pragma unroll
-          for (int u = 0; u < U; ++u) {
-            const int j = j0 + 8 * u;
-            dot[u] = 0.f;
-            if (j < nkb) {
-              const float* src = kb + static_cast<size_t>(j) * D;
-              if constexpr (DPL == 4) {
-                const float4 v = __ldg(reinterpret_cast<const float4*>(src));
-                dot[u] = fmaf(qv[0], v.x, fmaf(qv[1], v.y, fmaf(qv[2], v.z, qv[3] * v.w)));
-              } else {
-                const float2 v = __ldg(reinterpret_cast<const float2*>(src));
-                dot[u] = fmaf(qv[0], v.x, qv[1] * v.y);
+              for (int k = 0; k < 4; ++k) {
+                a[2 * k] += __uint_as_float(wv[k] << 16);
+                a[2 * k + 1] += __uint_as_float(wv[k] & 0xffff0000u);
               }
             }
           }
+          float* part = s_sbar;  // [RG][D]
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-#pragma unroll
-            for (int u = 0; u < U; ++u) dot[u] += __shfl_xor_sync(0xffffffffu, dot[u], o);
+          for (int k = 0; k < 8; ++k) part[rg * D + c8 * 8 + k] = a[k];
+          named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
+          if (st < D) {
+            float q = 0.f;
+#pragma unroll 8
+            for (int k = 0; k < RG; ++k) q += part[k * D + st];
+            s_qbar[st] = q / static_cast<float>(m_i);
           }
+          named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
+        }
+
+        // (1b) proxy scores s_bar_j (shared memory only) and their max; 8 warps, 16 rows in flight
+        // each (the pooled keys come from L2, so the loop is bound by how many loads are in flight)
+        {
+          constexpr int DPL = D / 32;
+          constexpr int U = 16;
+          float qv[DPL];
 #pragma unroll
-          for (int u = 0; u < U; ++u) {
-            const int j = j0 + 8 * u;
-            if (j < nkb) {
-              const float sc = dot[u] * p.inv_sqrt_d;
-              if (lane == 0) s_sbar[j] = sc;
-              wmax = fmaxf(wmax, sc);
+          for (int k = 0; k < DPL; ++k) qv[k] = s_qbar[lane * DPL + k];
+          const float* kb = p.kbar + static_cast<size_t>(bh) * nkb * D + lane * DPL;
+          float wmax = -INFINITY;
+          for (int j0 = sw; j0 < nkb; j0 += 8 * U) {
+            float dot[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+              const int j = j0 + 8 * u;
+              dot[u] = 0.f;
+              if (j < nkb) {
+                const float* src = kb + static_cast<size_t>(j) * D;
+                if constexpr (DPL == 4) {
+                  const float4 v = __ldg(reinterpret_cast<const float4*>(src));
+                  dot[u] = fmaf(qv[0], v.x, fmaf(qv[1], v.y, fmaf(qv[2], v.z, qv[3] * v.w)));
+                } else {
+                  const float2 v = __ldg(reinterpret_cast<const float2*>(src));
+                  dot[u] = fmaf(qv[0], v.x, qv[1] * v.y);
+                }
+              }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+              for (int u = 0; u < U; ++u) dot[u] += __shfl_xor_sync(0xffffffffu, dot[u], o);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+              const int j = j0 + 8 * u;
+              if (j < nkb) {
+                const float sc = dot[u] * p.inv_sqrt_d;
+                if (lane == 0) s_sbar[j] = sc;
+                wmax = fmaxf(wmax, sc);
+              }
             }
           }
+          if (lane == 0) s_red[sw] = wmax;
+          named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
         }
-        if (lane == 0) s_red[sw] = wmax;
-        named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
-      }
 
-      // (1c) keep bits (each warp ballots whole words), their prefix counts (warp 0), then the kept
-      // list and the pooled-tile list
-      {
-        float M = s_red[0];
+        // (1c) keep bits, each warp ballots whole words
+        {
+          float M = s_red[0];
 #pragma unroll
-        for (int k = 1; k < 8; ++k) M = fmaxf(M, s_red[k]);
-        const float thr = M - p.tau[bh % p.H];
-        const int nwords = (nkb + 31) / 32;
-        for (int i = sw; i < nwords; i += 8) {
-          const int j = 32 * i + lane;
-          const bool k = j < nkb && (s_sbar[j] >= thr || j < p.n_force);
-          const uint32_t m = __ballot_sync(0xffffffffu, k);
-          if (lane == 0) s_bits[i] = m;
+          for (int k = 1; k < 8; ++k) M = fmaxf(M, s_red[k]);
+          const float thr = M - p.tau[bh % p.H];
+          for (int i = sw; i < nwords; i += 8) {
+            const int j = 32 * i + lane;
+            const bool k = j < nkb && (s_sbar[j] >= thr || j < p.n_force);
+            const uint32_t m = __ballot_sync(0xffffffffu, k);
+            if (lane == 0) s_bits[i] = m;
+          }
         }
-        named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
+      }  // routed in this kernel
+      named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
+
+      // (1d) prefix counts of the keep words and the pooled-tile list (warp 0), then the kept list
+      {
         int* s_pref = reinterpret_cast<int*>(s_qbar + D);  // [kMaxKeyBlocks / 32]: kept blocks before word i
         if (sw == 0) {
           int run = 0;
@@ -507,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) {
             s_misc[MISC_NK] = alive ? nk : 0;
             s_misc[MISC_NC] = alive ? nc : 0;
-            atomicAdd(&p.ws[WS_COUNTS + bh], static_cast<uint32_t>(nk));
+            if (p.bits == nullptr) atomicAdd(&p.ws[WS_COUNTS + bh], static_cast<uint32_t>(nk));
           }
         }
         named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
@@ -518,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
       if (st == 0 && alive) mbar_arrive(bar_list);
-      if (p.kept_mask != nullptr) {
+      if (p.kept_mask != nullptr && p.bits == nullptr) {
         uint8_t* mrow = p.kept_mask + (static_cast<size_t>(bh) * p.nqb + qb) * nkb;
         for (int j = st; j < nkb; j += kSoftmaxThreads)
           mrow[j] = static_cast<uint8_t>((s_bits[j >> 5] >> (j & 31)) & 1u);
@@ -736,6 +748,7 @@ cudaError_t launch_tc_t(const FwdArgs& a, const CUtensorMap* maps, cudaStream_t 
   using C = TcCfg<D>;
   TcParams p;
   p.kbar = a.kbar;
+  p.bits = a.route_bits;
   p.O = static_cast<__nv_bfloat16*>(a.O);
   p.kept_mask = a.kept_mask;
   p.density = a.density;

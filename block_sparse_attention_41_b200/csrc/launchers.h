@@ -26,11 +26,17 @@ struct FwdArgs {
   uint32_t* ws;
   int num_sms;
   int drop_one_load;       // failure-detection test hook (bf16 path)
+  uint32_t* route_bits;    // bf16 path: [B*H, N_qb, ceil(N_kb/32)] keep bits from launch_route, or null
+                           // (the fused kernel then routes each unit itself)
   uint64_t wait_limit_ns;  // bound on every on-device wait
 };
 
 cudaError_t launch_pool(const void* K, const void* V, bool bf16, int BH, int L, int d, int block,
                         float* kbar, float* vbar, void* kbar_lp, void* vbar_lp, cudaStream_t stream);
+
+// bf16, d in {64, 128}, block 128: routing pass for every unit; writes a.route_bits, the optional
+// mask and the per-head kept counts (ws + WS_COUNTS).
+cudaError_t launch_route(const FwdArgs& a, cudaStream_t stream);
 
 // bf16, d in {64, 128}, block 128: TMA + tcgen05 persistent kernel.
 cudaError_t launch_fwd_tc(const FwdArgs& a, const CUtensorMap* maps /* Q, K, V, Kbar_lp, Vbar_lp */,

@@ -86,6 +86,18 @@ sol_status make_map(CUtensorMap* m, const void* base, int d, int rows, int BH) {
 
 bool size_ok(long long v, long long lim) { return v >= 1 && v <= lim; }
 
+// Workspace layout: [error, where, counter, done, counts[B*H]] rounded to 256 B (the header), then
+// the keep bits of the routing pass, u32[B*H][N_qb][ceil(N_kb/32)].
+size_t ws_header_bytes(int B, int H) {
+  const size_t words = static_cast<size_t>(sol::WS_COUNTS) + static_cast<size_t>(B) * H;
+  return (words * 4 + 255) / 256 * 256;
+}
+size_t ws_bits_bytes(int B, int H, int L, int block) {
+  const size_t nb = (static_cast<size_t>(L) + block - 1) / block;
+  const size_t bytes = static_cast<size_t>(B) * H * nb * ((nb + 31) / 32) * 4;
+  return (bytes + 255) / 256 * 256;
+}
+
 // ---- workspace in the library's own device memory, for sol_attn_fwd_noalloc -------------------
 constexpr int kNoAllocMaxHeads = 4096;  // B * H
 constexpr size_t kNoAllocWords = static_cast<size_t>(sol::WS_COUNTS) + kNoAllocMaxHeads;
@@ -170,11 +182,8 @@ sol_status sol_attn_pool(const void* K, const void* V, sol_dtype dt, int B, int 
 }
 
 size_t sol_attn_fwd_workspace_bytes(int B, int H, int L, int block_q) {
-  (void)L;
-  (void)block_q;
-  if (B < 1 || H < 1) return 0;
-  const size_t words = static_cast<size_t>(sol::WS_COUNTS) + static_cast<size_t>(B) * H;
-  return (words * 4 + 255) / 256 * 256;
+  if (B < 1 || H < 1 || L < 1 || block_q < 1) return 0;
+  return ws_header_bytes(B, H) + ws_bits_bytes(B, H, L, block_q);
 }
 
 sol_status sol_attn_fwd(const void* Q, const void* K, const void* V, const float* kbar, const float* vbar,
@@ -214,8 +223,10 @@ sol_status sol_attn_fwd(const void* Q, const void* K, const void* V, const float
   if (n_force < 0 || n_force > nkb) return fail(SOL_EINVAL, "n_force=%d must be in [0, N_kb=%lld]", n_force, nkb);
   if (static_cast<long long>(B) * H * nkb >= (1ll << 31)) return fail(SOL_EUNSUPPORTED, "B*H*N_qb must be < 2^31");
   if (static_cast<long long>(B) * H > 65535) return fail(SOL_EUNSUPPORTED, "B*H must be <= 65535");
-  const size_t need = sol_attn_fwd_workspace_bytes(B, H, L, block_q);
+  const size_t need = ws_header_bytes(B, H);
   if (ws_bytes < need) return fail(SOL_EINVAL, "workspace too small (%zu < %zu bytes)", ws_bytes, need);
+  // a workspace that also holds the keep bits gets the separate routing pass (bf16 path)
+  const bool route_pass = bf16 && ws_bytes >= need + ws_bits_bytes(B, H, L, block_q);
 
   int sms = 0;
   sol_status st = current_device(&sms);
@@ -251,6 +262,7 @@ sol_status sol_attn_fwd(const void* Q, const void* K, const void* V, const float
   a.num_sms = sms;
   a.drop_one_load = 0;
   a.wait_limit_ns = 2000000000ull;
+  a.route_bits = route_pass ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + need) : nullptr;
 
   if (bf16) {
     a.drop_one_load = g_drop_one_load;
@@ -263,6 +275,10 @@ sol_status sol_attn_fwd(const void* Q, const void* K, const void* V, const float
     if ((st = make_map(&maps[2], V, d, L, B * H)) != SOL_OK) return st;
     if ((st = make_map(&maps[3], kbar_lp, d, nkb_i, B * H)) != SOL_OK) return st;
     if ((st = make_map(&maps[4], vbar_lp, d, nkb_i, B * H)) != SOL_OK) return st;
+    if (route_pass) {
+      e = sol::launch_route(a, s);
+      if (e != cudaSuccess) return cuda_fail(e, "routing launch");
+    }
     e = sol::launch_fwd_tc(a, maps, s);
     if (e != cudaSuccess) return cuda_fail(e, "tcgen05 forward launch");
   } else {

@@ -78,12 +78,19 @@ sol_status sol_attn_pool(const void* K, const void* V, sol_dtype dt, int B, int 
                          void* stream);
 
 /* Bytes of device workspace sol_attn_fwd needs for this problem. The workspace holds the
- * persistent scheduler's work counter, the per-(b,h) kept-block counters and the sticky
- * device error word. Zero it once after allocation; later calls keep it consistent. */
+ * persistent scheduler's work counter, the per-(b,h) kept-block counters and the sticky device
+ * error word (a header of 4 * (4 + B*H) bytes rounded up to 256), followed by the keep bits of the
+ * routing pass: B*H*N_qb*ceil(N_kb/32) 32-bit words, rounded up to 256 bytes (1.8 MB for
+ * B=1, H=40, L=75600, block 128). Zero it once after allocation; later calls keep it consistent. */
 size_t sol_attn_fwd_workspace_bytes(int B, int H, int L, int block_q);
 
-/* The fused forward: routing, exact attention on kept blocks, skipped-block correction and the
- * epilogue, in one kernel launch (Sol-Attn project page, Abstract).
+/* The forward: routing, exact attention on kept blocks, skipped-block correction and the epilogue
+ * (Sol-Attn project page, Abstract). For SOL_BF16 with a workspace of the full size returned above,
+ * routing runs as its own pass first. That pass routes 4-16 query blocks of one head per CTA, so
+ * each head's pooled keys are read once per group of query blocks instead of once per block. It
+ * writes only the keep bits into the workspace, then the fused kernel turns them into its tile
+ * lists. With a workspace that holds only the header, the fused kernel routes each query block
+ * itself, with the same fp32 arithmetic in the same order, so both paths keep the same blocks.
  *
  *   Q, K, V     device, [B, H, L, d] in dtype `dt`
  *   kbar        device, float32 [B, H, N_kb, d] from sol_attn_pool: the routing proxy
@@ -100,9 +107,12 @@ size_t sol_attn_fwd_workspace_bytes(int B, int H, int L, int block_q);
  *   kept_mask   device, uint8 [B, H, N_qb, N_kb] or NULL: 1 where block j was kept for query
  *               block i
  *   density     device, float32 [B, H] or NULL: kept blocks / (N_qb * N_kb) per head
- *   workspace   device, >= sol_attn_fwd_workspace_bytes(...) bytes, zeroed once after allocation
+ *   workspace   device, zeroed once after allocation: sol_attn_fwd_workspace_bytes(...) bytes, or
+ *               at least its header (4 * (4 + B*H) bytes rounded up to 256), which selects routing
+ *               inside the fused kernel; smaller returns SOL_EINVAL
  * Limits: H <= 256, N_kb <= 4096, B*H*N_qb < 2^31.
- * The proxy scores s_bar stay in shared memory and are never written to global memory.
+ * The proxy scores s_bar stay in shared memory and are never written to global memory; only the
+ * keep bits are.
  */
 sol_status sol_attn_fwd(const void* Q, const void* K, const void* V, const float* kbar,
                         const float* vbar, const void* kbar_lp, const void* vbar_lp,
