@@ -393,11 +393,14 @@ def run_ours(args, w):
                        "parallelism": f"replica x{world}"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": achieved / pk["bf16_tflops"], "traffic": traffic,
-                         "kernel": "sol_fwd_tc_kernel", "fwd_ms": fwd_ms,
+                         "kernel": "sol_fwd_tc_kernel",
+                         "timed": "one sol_attn_fwd call: routing pass + fused kernel (the fused kernel alone is "
+                                  "faster; the ncu launch list gives the split)",
+                         "fwd_ms": fwd_ms,
                          "peak_source": f"{pk['source']} bf16 dense (burst)"},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": 3 * args.steps,  # pool, routing pass, fused forward
             "clocks": clocks,
             "sweep": sweep,
         }

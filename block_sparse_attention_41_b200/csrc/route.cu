@@ -34,6 +34,33 @@ struct RouteParams {
   float tau[kMaxHeads];
 };
 
+// Sum each of the N values of a lane over the 32 lanes, with N - 1 + (5 - log2 N) shuffles instead
+// of 5 N: at every butterfly step a lane keeps half of its values and receives the partner's
+// copies of that half, until one value is left. The additions follow the same pairwise tree as
+// the plain xor reduction (a lane adds its own value and its partner's at every level), so the
+// sums are bit-identical to it. On return v[0] holds the total of value r = lane >> (5 - log2 N):
+// the first step decides the top bit of r from lane bit 4, the next from lane bit 3, and so on.
+template <int N, int O = 16>
+__device__ __forceinline__ void butterfly_sum(float (&v)[N], int lane) {
+  if constexpr (O >= 1) {
+    if constexpr (N > 1) {
+      constexpr int H = N / 2;
+      const bool hi = (lane & O) != 0;
+#pragma unroll
+      for (int k = 0; k < H; ++k) {
+        const float send = hi ? v[k] : v[H + k];
+        const float keep = hi ? v[H + k] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+      }
+      float (&w)[H] = *reinterpret_cast<float (*)[H]>(&v[0]);
+      butterfly_sum<H, O / 2>(w, lane);
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], O);
+      butterfly_sum<1, O / 2>(v, lane);
+    }
+  }
+}
+
 template <int D, int R>
 __global__ void __launch_bounds__(kRouteThreads) sol_route_kernel(const __grid_constant__ RouteParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -48,37 +75,55 @@ __global__ void __launch_bounds__(kRouteThreads) sol_route_kernel(const __grid_c
   const int nkb = p.nkb;
   if (tid == 0) s_cnt = 0;
 
-  // (1) q_bar of each of the nr query blocks: thread t sums a 16-byte chunk (8 columns) over a
-  // strided set of rows; partial sums meet in shared memory
+  // (1) q_bar of each of the nr query blocks, four blocks at a time: thread t sums a 16-byte chunk
+  // (8 columns) of each over a strided set of rows (the same rows, in the same order, as the fused
+  // kernel's own routing); partial sums meet in shared memory
   {
     constexpr int CH = D / 8;
     constexpr int RG = kRouteThreads / CH;
+    constexpr int NB = 4;
     const int c8 = tid % CH, rg = tid / CH;
-    float* part = s_sc;  // [RG][D]
-    for (int r = 0; r < nr; ++r) {
-      const int row0 = (qb0 + r) * kRows;
-      const int m = min(kRows, p.L - row0);
-      const __nv_bfloat16* qrow = p.Q + (static_cast<size_t>(bh) * p.L + row0) * D + c8 * 8;
-      float a[8];
+    float* part = s_sc;  // [NB][RG][D]
+    for (int r0 = 0; r0 < nr; r0 += NB) {
+      float a[NB][8];
+      int m[NB];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) a[k] = 0.f;
-#pragma unroll 4
-      for (int rr = rg; rr < m; rr += RG) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(qrow + static_cast<size_t>(rr) * D));
-        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+      for (int rb = 0; rb < NB; ++rb) {
+        m[rb] = (r0 + rb < nr) ? min(kRows, p.L - (qb0 + r0 + rb) * kRows) : 0;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          a[2 * k] += __uint_as_float(wv[k] << 16);
-          a[2 * k + 1] += __uint_as_float(wv[k] & 0xffff0000u);
+        for (int k = 0; k < 8; ++k) a[rb][k] = 0.f;
+      }
+      const __nv_bfloat16* qrow = p.Q + (static_cast<size_t>(bh) * p.L + static_cast<size_t>(qb0 + r0) * kRows) * D + c8 * 8;
+#pragma unroll 2
+      for (int rr = rg; rr < kRows; rr += RG) {
+        uint4 v[NB];
+#pragma unroll
+        for (int rb = 0; rb < NB; ++rb)
+          if (rr < m[rb]) v[rb] = __ldg(reinterpret_cast<const uint4*>(qrow + static_cast<size_t>(rb * kRows + rr) * D));
+#pragma unroll
+        for (int rb = 0; rb < NB; ++rb) {
+          if (rr < m[rb]) {
+            const uint32_t wv[4] = {v[rb].x, v[rb].y, v[rb].z, v[rb].w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              a[rb][2 * k] += __uint_as_float(wv[k] << 16);
+              a[rb][2 * k + 1] += __uint_as_float(wv[k] & 0xffff0000u);
+            }
+          }
         }
       }
 #pragma unroll
-      for (int k = 0; k < 8; ++k) part[rg * D + c8 * 8 + k] = a[k];
+      for (int rb = 0; rb < NB; ++rb)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) part[(rb * RG + rg) * D + c8 * 8 + k] = a[rb][k];
       __syncthreads();
-      if (tid < D) {
-        float q = 0.f;
-        for (int k = 0; k < RG; ++k) q += part[k * D + tid];
-        s_qbar[r * D + tid] = q / static_cast<float>(m);
+      for (int idx = tid; idx < NB * D; idx += kRouteThreads) {
+        const int rb = idx / D, c = idx % D;
+        if (r0 + rb < nr) {
+          float q = 0.f;
+          for (int k = 0; k < RG; ++k) q += part[(rb * RG + k) * D + c];
+          s_qbar[(r0 + rb) * D + c] = q / static_cast<float>(m[rb]);
+        }
       }
       __syncthreads();
     }
@@ -88,7 +133,7 @@ __global__ void __launch_bounds__(kRouteThreads) sol_route_kernel(const __grid_c
   {
     constexpr int DPL = D / 32;
     const float* kb = p.kbar + static_cast<size_t>(bh) * nkb * D + lane * DPL;
-    constexpr int U = 2;  // key blocks in flight per warp
+    constexpr int U = 4;  // key blocks in flight per warp
     for (int j0 = warp; j0 < nkb; j0 += kRouteWarps * U) {
       float kv[U][DPL];
 #pragma unroll
@@ -114,22 +159,19 @@ __global__ void __launch_bounds__(kRouteThreads) sol_route_kernel(const __grid_c
         for (int r = 0; r < R; ++r) {
           // the same fp32 operation order as the fused kernel's own routing, so both give the
           // same keep bits
-          const float* qv = s_qbar + r * D + lane * DPL;
-          if constexpr (DPL == 4)
-            dot[r] = fmaf(qv[0], kv[u][0], fmaf(qv[1], kv[u][1], fmaf(qv[2], kv[u][2], qv[3] * kv[u][3])));
-          else
-            dot[r] = fmaf(qv[0], kv[u][0], qv[1] * kv[u][1]);
+          if constexpr (DPL == 4) {
+            const float4 qv = *reinterpret_cast<const float4*>(s_qbar + r * D + lane * DPL);
+            dot[r] = fmaf(qv.x, kv[u][0], fmaf(qv.y, kv[u][1], fmaf(qv.z, kv[u][2], qv.w * kv[u][3])));
+          } else {
+            const float2 qv = *reinterpret_cast<const float2*>(s_qbar + r * D + lane * DPL);
+            dot[r] = fmaf(qv.x, kv[u][0], qv.y * kv[u][1]);
+          }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-#pragma unroll
-          for (int r = 0; r < R; ++r) dot[r] += __shfl_xor_sync(0xffffffffu, dot[r], o);
-        }
-        if (lane == 0 && j < nkb) {
-#pragma unroll
-          for (int r = 0; r < R; ++r)
-            if (r < nr) s_sc[r * nkb + j] = dot[r] * p.inv_sqrt_d;
-        }
+        butterfly_sum<R>(dot, lane);
+        // lane l now holds the total of query block r(l); the lanes that agree on r hold the same value
+        constexpr int LOGR = R == 16 ? 4 : (R == 8 ? 3 : 2);
+        const int r = lane >> (5 - LOGR);
+        if ((lane & ((32 >> LOGR) - 1)) == 0 && j < nkb && r < nr) s_sc[r * nkb + j] = dot[0] * p.inv_sqrt_d;
       }
     }
   }
@@ -182,9 +224,8 @@ cudaError_t launch_route_t(const FwdArgs& a, cudaStream_t stream) {
   p.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   for (int h = 0; h < kMaxHeads; ++h) p.tau[h] = h < a.H ? a.tau[h] : 0.f;
   constexpr int RG = kRouteThreads / (D / 8);
-  const size_t sc_floats = static_cast<size_t>(R) * p.nkb > static_cast<size_t>(RG) * D
-                               ? static_cast<size_t>(R) * p.nkb
-                               : static_cast<size_t>(RG) * D;
+  const size_t part_floats = static_cast<size_t>(4) * RG * D;  // q_bar partial sums of four blocks
+  const size_t sc_floats = static_cast<size_t>(R) * p.nkb > part_floats ? static_cast<size_t>(R) * p.nkb : part_floats;
   const size_t smem = (static_cast<size_t>(R) * D + sc_floats) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(sol_route_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));

@@ -46,6 +46,10 @@ def test_workspace_size(lib):
     n = sa.sol_attn_fwd_workspace_bytes(2, 32, 33272, 128)
     assert n % 256 == 0 and n >= 4 * (4 + 64)
     assert sa.sol_attn_fwd_workspace_bytes(0, 1, 1, 1) == 0
+    # header (error, where, counter, done, 40 per-head counts) + keep bits 40 x 591 x ceil(591/32) words
+    header = ((4 + 40) * 4 + 255) // 256 * 256
+    bits = -(-(40 * 591 * 19 * 4) // 256) * 256
+    assert sa.sol_attn_fwd_workspace_bytes(1, 40, 75600, 128) == header + bits
 
 
 # fake, 16-byte aligned device addresses: validation must reject before any of them is used

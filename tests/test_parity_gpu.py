@@ -239,6 +239,53 @@ def test_bf16_identical_block_keys_give_dense_attention():
     assert err.max() <= TOL_BF16_MAX and err.mean() <= TOL_BF16_MEAN
 
 
+# ------------------------------------------------------------------------------------------------
+# routing pass (full workspace) against the fused kernel's own routing (header-only workspace)
+# ------------------------------------------------------------------------------------------------
+
+def _header_only_workspace(B, H, device):
+    return torch.zeros(((4 + B * H) * 4 + 255) // 256 * 256, dtype=torch.uint8, device=device)
+
+
+@pytest.mark.parametrize("L,d,H", [(3000, 128, 3), (1500, 64, 2), (262_221, 128, 1), (524_288, 64, 1)])
+def test_routing_pass_matches_in_kernel_routing(L, d, H):
+    """Both routing paths do the same fp32 arithmetic in the same order, so the mask, the density
+    and O agree bit for bit. N_kb = 2049 and 4096 (the limit) run the routing pass with 4 query
+    blocks per CTA; sampled query blocks of those are also checked against the oracle."""
+    Qh, Kh, Vh = local_inputs(1, H, L, d, seed=L % 997 + d)
+    Q, K, V = (torch.from_numpy(x).to(torch.bfloat16).cuda() for x in (Qh, Kh, Vh))
+    kbar, vbar, klp, vlp = sa.sol_attn_pool(K, V, 128)
+    nb = -(-L // 128)
+    tau = {1: [0.3], 2: [0.4, 1.2], 3: [0.0, 1.0, math.inf]}[H]
+    outs = []
+    for ws in (sa.new_workspace(1, H, L, 128, Q.device), _header_only_workspace(1, H, Q.device)):
+        mask = torch.empty((1, H, nb, nb), dtype=torch.uint8, device="cuda")
+        dens = torch.empty((1, H), dtype=torch.float32, device="cuda")
+        O = sa.sol_attn_fwd(Q, K, V, kbar, vbar, klp, vlp, tau, 128, 128, kept_mask=mask, density=dens, workspace=ws)
+        sa.sol_attn_check_device_error(ws)
+        outs.append((O, mask, dens))
+    assert torch.equal(outs[0][1], outs[1][1])
+    assert torch.equal(outs[0][2], outs[1][2])
+    assert torch.equal(outs[0][0], outs[1][0])
+    O, mask, dens = outs[0]
+    check_mask_density(mask, dens)
+    if nb <= 64:
+        st = full_compare(Qh, Kh, Vh, O, mask, tau, 128)
+    else:
+        units = sorted(set(np.random.default_rng(d).choice(nb, size=3, replace=False).tolist()) | {0, nb - 1})
+        mk = mask.cpu().numpy().astype(bool)[0, 0]
+        O_ref, keep, sbar, M = oracle.forward_head(Qh[0, 0], Kh[0, 0], Vh[0, 0], tau[0], 128, 128, 0, units=units,
+                                                   keep_override=mk)
+        band = oracle.band_mask(sbar[units], M[units], tau[0], 0)
+        rows = np.concatenate([np.arange(i * 128, min(L, i * 128 + 128)) for i in units])
+        e = np.abs(O[0, 0].double().cpu().numpy()[rows] - O_ref[rows])
+        st = {"max_abs": float(e.max()), "mean_abs": float(e.mean()),
+              "mask_mismatch_outside_band": int((mk[units][~band] != keep[units][~band]).sum()),
+              "band_entries": int(band.sum()), "units": len(units)}
+    report(f"routing pass L={L} d={d}", st)
+    check_bf16(st)
+
+
 @pytest.mark.parametrize("blk,d", [(32, 32), (64, 64), (128, 128), (64, 128)])
 def test_f32_path_shapes(blk, d):
     Qh, Kh, Vh = local_inputs(1, 2, 700, d, seed=blk + d, dtype="f32")
