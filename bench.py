@@ -188,6 +188,61 @@ def oracle_sample(w, tau, budget_s: float, max_units: int = 64, seed_offset: int
     return kept_tiles, elapsed, done, threads
 
 
+def measure_qknorm_rope_pool(w, Q, K, V, stream, pk, cpu_ok, max_over_ranks, barrier, world):
+    """The fused QK-norm + RoPE + pooling step on the workload's own Q, K, V (standing in for the
+    raw projections): CUDA-event time of the kernel alone, HBM roofline, and the oracle timed on a
+    bounded host sample."""
+    import torch
+    from block_sparse_attention_41_b200 import sol_attn as sa
+    d, blk, nb = w.d, w.block, w.n_blocks
+    cos, sin = wl.rope_tables(w.grid, d)
+    gq, gk = wl.qk_norm_gains(d, w.seed)
+    dev = Q.device
+    tc, ts, tq, tk = (torch.from_numpy(np.ascontiguousarray(a)).to(dev) for a in (cos, sin, gq, gk))
+    Qo, Ko = torch.empty_like(Q), torch.empty_like(K)
+    kb = torch.empty((w.B, w.H, nb, d), dtype=torch.float32, device=dev)
+    vb = torch.empty_like(kb)
+    kl = torch.empty((w.B, w.H, nb, d), dtype=torch.bfloat16, device=dev)
+    vl = torch.empty_like(kl)
+
+    def run():
+        sa.sol_attn_qknorm_rope_pool(Q, K, V, tq, tk, tc, ts, blk, 1e-6, Qo, Ko, kb, vb, kl, vl, stream=stream)
+
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    barrier()
+    n_it = 10
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_it):
+        run()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1)) / n_it
+    elem_bytes = Q.numel() * Q.element_size()
+    pooled = 2 * w.B * w.H * nb * d * (4 + 2)
+    alg = 5 * elem_bytes + 2 * w.L * (d // 2) * 4 + 2 * d * 4 + pooled  # Q,K,V read; Q',K' written; tables
+    gbs = alg / (ms * 1e-3) / 1e9
+    out = {"kernel": "sol_qknorm_rope_pool_kernel", "ms": ms, "algorithmic_bytes": alg,
+           "unfused_bytes": alg + elem_bytes, "GB/s": world * gbs, "bound": "hbm", "peak_GB/s": pk["hbm_gbs"],
+           "frac": gbs / pk["hbm_gbs"],
+           "note": "norm+RoPE then a separate pool would read the stored keys once more (unfused_bytes)"}
+    del Qo, Ko, kb, vb, kl, vl
+    if cpu_ok:
+        import oracle
+        q, k, v = (x.astype(np.float64) for x in wl.head_tensors(w, 0, 0))
+        rows = min(w.L, 64 * blk)
+        t0 = time.perf_counter()
+        oracle.qknorm_rope_pool_head(q[:rows], k[:rows], v[:rows], gq, gk, cos[:rows], sin[:rows], 1e-6, blk,
+                                     lambda x: wl.round_to_bf16(x).astype(np.float64))
+        secs = time.perf_counter() - t0
+        sample_bytes = alg * rows / (w.B * w.H * w.L)
+        out["cpu_baseline"] = {"value": sample_bytes / secs / 1e9, "unit": "GB/s", "kind": "oracle",
+                               "sample": f"{rows} tokens of one head ({secs:.2f} s of float64 oracle work)"}
+    return out
+
+
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -339,6 +394,12 @@ def run_ours(args, w):
             for s in sweep:
                 s["speedup_vs_dense"] = dense[0]["ms_per_step"] / s["ms_per_step"]
 
+    next_rows = None
+    if not args.no_next and w.dtype == "bf16" and w.n_text == 0:
+        next_rows = {"qknorm_rope_pool": measure_qknorm_rope_pool(
+            w, Q, K, V, stream, pk, rank == 0 and world == 1 and not args.no_cpu_baseline, max_over_ranks, barrier,
+            world)}
+
     # end to end through the public API: pinned host inputs in, host output back, every step
     e2e = None
     if not args.no_e2e:
@@ -403,6 +464,7 @@ def run_ours(args, w):
             "gpu_launches": 3 * args.steps,  # pool, routing pass, fused forward
             "clocks": clocks,
             "sweep": sweep,
+            "next_rows": next_rows,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -430,6 +492,7 @@ def main():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next", action="store_true", help="skip the fused QK-norm + RoPE + pooling measurement")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-budget", type=float, default=0.0,
                     help="reference arm: seconds of oracle work per step (default: fit a few minutes)")

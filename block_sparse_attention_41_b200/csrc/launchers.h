@@ -34,6 +34,27 @@ struct FwdArgs {
 cudaError_t launch_pool(const void* K, const void* V, bool bf16, int BH, int L, int d, int block,
                         float* kbar, float* vbar, void* kbar_lp, void* vbar_lp, cudaStream_t stream);
 
+struct RopePoolArgs {
+  const void* Q;  // bf16 [BH, L, d]
+  const void* K;
+  const void* V;
+  const float* gain_q;  // [d]
+  const float* gain_k;  // [d]
+  const float* cos;     // [L, d/2]
+  const float* sin;     // [L, d/2]
+  float eps;
+  void* Qout;  // bf16 [BH, L, d]
+  void* Kout;
+  float* kbar;  // fp32 [BH, N_kb, d]
+  float* vbar;
+  void* kbar_lp;  // bf16 [BH, N_kb, d]
+  void* vbar_lp;
+  int BH, L, d, block;
+};
+
+// bf16, d in {64, 128}: QK RMS norm + rotary embedding + K/V block pooling in one pass.
+cudaError_t launch_qknorm_rope_pool(const RopePoolArgs& a, cudaStream_t stream);
+
 // bf16, d in {64, 128}, block 128: routing pass for every unit; writes a.route_bits, the optional
 // mask and the per-head kept counts (ws + WS_COUNTS).
 cudaError_t launch_route(const FwdArgs& a, cudaStream_t stream);

@@ -181,6 +181,50 @@ sol_status sol_attn_pool(const void* K, const void* V, sol_dtype dt, int B, int 
   return SOL_OK;
 }
 
+sol_status sol_attn_qknorm_rope_pool(const void* Q, const void* K, const void* V, const float* gain_q,
+                                     const float* gain_k, const float* rope_cos, const float* rope_sin, float eps,
+                                     int B, int H, int L, int d, int block_k, void* Q_out, void* K_out, float* kbar,
+                                     float* vbar, void* kbar_lp, void* vbar_lp, void* stream) {
+  g_last_error.clear();
+  if (!size_ok(B, 1 << 16) || !size_ok(H, 1 << 16) || !size_ok(L, 1 << 28) || !size_ok(d, 1 << 16) ||
+      !size_ok(block_k, 1 << 20))
+    return fail(SOL_EINVAL, "sizes must be positive (B=%d H=%d L=%d d=%d block_k=%d)", B, H, L, d, block_k);
+  if (!(eps > 0.f) || std::isinf(eps)) return fail(SOL_EINVAL, "eps=%g must be positive and finite", eps);
+  const void* ptrs[] = {Q, K, V, gain_q, gain_k, rope_cos, rope_sin, Q_out, K_out, kbar, vbar, kbar_lp, vbar_lp};
+  for (const void* ptr : ptrs) {
+    if (ptr == nullptr) return fail(SOL_EINVAL, "every pointer argument must be non-null");
+    if (!aligned16(ptr)) return fail(SOL_EINVAL, "device pointers must be 16-byte aligned");
+  }
+  if (d != 64 && d != 128) return fail(SOL_EUNSUPPORTED, "QK-norm + RoPE + pooling needs d in {64, 128} (d=%d)", d);
+  if (block_k > 4096) return fail(SOL_EUNSUPPORTED, "block_k must be <= 4096");
+  if (static_cast<long long>(B) * H > 65535) return fail(SOL_EUNSUPPORTED, "B*H must be <= 65535");
+  int sms = 0;
+  sol_status st = current_device(&sms);
+  if (st != SOL_OK) return st;
+  sol::RopePoolArgs a;
+  a.Q = Q;
+  a.K = K;
+  a.V = V;
+  a.gain_q = gain_q;
+  a.gain_k = gain_k;
+  a.cos = rope_cos;
+  a.sin = rope_sin;
+  a.eps = eps;
+  a.Qout = Q_out;
+  a.Kout = K_out;
+  a.kbar = kbar;
+  a.vbar = vbar;
+  a.kbar_lp = kbar_lp;
+  a.vbar_lp = vbar_lp;
+  a.BH = B * H;
+  a.L = L;
+  a.d = d;
+  a.block = block_k;
+  cudaError_t e = sol::launch_qknorm_rope_pool(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "QK-norm + RoPE + pooling launch");
+  return SOL_OK;
+}
+
 size_t sol_attn_fwd_workspace_bytes(int B, int H, int L, int block_q) {
   if (B < 1 || H < 1 || L < 1 || block_q < 1) return 0;
   return ws_header_bytes(B, H) + ws_bits_bytes(B, H, L, block_q);

@@ -30,6 +30,7 @@ EXPORTED = (
     "sol_attn_check_device_error",
     "sol_attn_debug_drop_one_load",
     "sol_attn_fwd_noalloc",
+    "sol_attn_qknorm_rope_pool",
 )
 
 
@@ -69,6 +70,9 @@ def load_library() -> ctypes.CDLL:
     lib.sol_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, f32p, i32, i32, i32, i32, i32, i32, i32, i32,
                                          vp, vp, vp, vp]
     lib.sol_attn_fwd_noalloc.restype = i32
+    lib.sol_attn_qknorm_rope_pool.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, i32, i32, i32, i32,
+                                              vp, vp, vp, vp, vp, vp, vp]
+    lib.sol_attn_qknorm_rope_pool.restype = i32
     lib.sol_attn_check_device_error.argtypes = [vp, vp]
     lib.sol_attn_check_device_error.restype = i32
     lib.sol_attn_debug_drop_one_load.argtypes = [i32]
@@ -140,6 +144,36 @@ def sol_attn_pool(K: torch.Tensor, V: torch.Tensor, block_k: int, kbar=None, vba
                                       _ptr(kbar_lp), _ptr(vbar_lp), _stream(stream))
     _check(st, "sol_attn_pool")
     return kbar, vbar, kbar_lp, vbar_lp
+
+
+def sol_attn_qknorm_rope_pool(Q, K, V, gain_q, gain_k, rope_cos, rope_sin, block_k: int, eps: float = 1e-6,
+                              Q_out=None, K_out=None, kbar=None, vbar=None, kbar_lp=None, vbar_lp=None, stream=None):
+    """QK RMS norm + rotary embedding of Q and K, and the block means of the stored K and of V, in
+    one pass. Returns (Q_out, K_out, kbar, vbar, kbar_lp, vbar_lp). Pass Q_out=Q, K_out=K to
+    work in place."""
+    for n, t in (("Q", Q), ("K", K), ("V", V)):
+        _need_cuda(n, t, torch.bfloat16)
+    B, H, L, d = Q.shape
+    if K.shape != Q.shape or V.shape != Q.shape:
+        raise ValueError("Q, K and V must have the same shape [B, H, L, d]")
+    for n, t in (("gain_q", gain_q), ("gain_k", gain_k), ("rope_cos", rope_cos), ("rope_sin", rope_sin)):
+        _need_cuda(n, t, torch.float32)
+    if rope_cos.shape != (L, d // 2) or rope_sin.shape != (L, d // 2):
+        raise ValueError(f"rope tables must be [L, d/2] = [{L}, {d // 2}]")
+    nkb = -(-L // block_k)
+    dev = Q.device
+    Q_out = torch.empty_like(Q) if Q_out is None else Q_out
+    K_out = torch.empty_like(K) if K_out is None else K_out
+    kbar = torch.empty((B, H, nkb, d), dtype=torch.float32, device=dev) if kbar is None else kbar
+    vbar = torch.empty((B, H, nkb, d), dtype=torch.float32, device=dev) if vbar is None else vbar
+    kbar_lp = torch.empty((B, H, nkb, d), dtype=torch.bfloat16, device=dev) if kbar_lp is None else kbar_lp
+    vbar_lp = torch.empty((B, H, nkb, d), dtype=torch.bfloat16, device=dev) if vbar_lp is None else vbar_lp
+    st = load_library().sol_attn_qknorm_rope_pool(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(gain_q), _ptr(gain_k), _ptr(rope_cos), _ptr(rope_sin), ctypes.c_float(eps),
+        B, H, L, d, block_k, _ptr(Q_out), _ptr(K_out), _ptr(kbar), _ptr(vbar), _ptr(kbar_lp), _ptr(vbar_lp),
+        _stream(stream))
+    _check(st, "sol_attn_qknorm_rope_pool")
+    return Q_out, K_out, kbar, vbar, kbar_lp, vbar_lp
 
 
 def sol_attn_fwd_workspace_bytes(B: int, H: int, L: int, block_q: int) -> int:

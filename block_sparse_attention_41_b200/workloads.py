@@ -137,6 +137,35 @@ def positional_feature(grid: tuple, d: int) -> np.ndarray:
     return feat
 
 
+def rope_tables(grid: tuple, d: int, base: float = 10000.0):
+    """cos, sin float32 [T*Y*X, d/2] of 3-D rotary angles for the QK-norm + RoPE step's inputs.
+
+    The d/2 interleaved pairs are split over the axes (t, y, x): n_y = n_x = (d/2) // 3 pairs, the
+    rest to t. Pair j of an axis with n pairs turns by pos_axis * base^(-j/n). Tokens run
+    row-major over the grid, x fastest. These are inputs handed to the kernel and to the oracle.
+    """
+    T, Y, X = grid
+    n = T * Y * X
+    tok = np.arange(n)
+    pos = np.stack([tok // (Y * X), (tok // X) % Y, tok % X], axis=1).astype(np.float64)
+    half = d // 2
+    ny = half // 3
+    counts = (half - 2 * ny, ny, ny)
+    ang = np.empty((n, half), dtype=np.float64)
+    col = 0
+    for axis, cnt in enumerate(counts):
+        theta = base ** (-np.arange(cnt, dtype=np.float64) / cnt)
+        ang[:, col:col + cnt] = pos[:, axis:axis + 1] * theta[None, :]
+        col += cnt
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
+
+def qk_norm_gains(d: int, seed: int):
+    """Seeded RMS-norm gains (float32 [d] each) for queries and keys: 1 + N(0, 0.1^2)."""
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed, spawn_key=(99,))))
+    return tuple((1.0 + 0.1 * rng.standard_normal(d)).astype(np.float32) for _ in range(2))
+
+
 def round_to_bf16(x) -> np.ndarray:
     """float -> float32 (nearest even) -> bf16 (nearest even); returned as float32 values."""
     x32 = np.ascontiguousarray(x, dtype=np.float32)

@@ -77,6 +77,32 @@ sol_status sol_attn_pool(const void* K, const void* V, sol_dtype dt, int B, int 
                          int block_k, float* kbar, float* vbar, void* kbar_lp, void* vbar_lp,
                          void* stream);
 
+/* QK RMS norm + rotary embedding + block pooling in one pass: the step before the attention,
+ * which kernel fusion folds together (Sol-Engine README, "The five acceleration methods", kernel
+ * fusion of QK-norm + RoPE). The pages print no formula; this is the textbook form. For each
+ * (b, h) and token t, and for Q with gain_q and K with gain_k:
+ *   y  = x / sqrt(mean_c x_c^2 + eps) * gain          (RMS norm over the d head channels)
+ *   y' = each interleaved pair (y_2i, y_2i+1) turned by the angle with cosine rope_cos[t, i] and
+ *        sine rope_sin[t, i]:  (y_2i c - y_2i+1 s,  y_2i s + y_2i+1 c)
+ * y' goes to Q_out / K_out (bf16, nearest even). In the same pass, kbar/vbar (and their bf16
+ * mirrors) receive the block means of the STORED keys (after rounding) and of V. These are the
+ * same quantities sol_attn_pool computes from K_out and V, up to fp32 summation order. So K_out is
+ * not read back by a separate pooling pass.
+ *
+ *   Q, K, V          device, bf16 [B, H, L, d]
+ *   gain_q, gain_k   device, float32 [d]
+ *   rope_cos/sin     device, float32 [L, d/2] (the same for every b, h)
+ *   eps              > 0
+ *   Q_out, K_out     device, bf16 [B, H, L, d]; may be Q and K themselves (in place)
+ *   kbar, vbar       device, float32 [B, H, N_kb, d];  kbar_lp, vbar_lp: bf16 mirrors
+ * Supported: d in {64, 128}, 1 <= block_k <= 4096, B*H <= 65535. All pointers non-null and
+ * 16-byte aligned (else SOL_EINVAL). */
+sol_status sol_attn_qknorm_rope_pool(const void* Q, const void* K, const void* V, const float* gain_q,
+                                     const float* gain_k, const float* rope_cos, const float* rope_sin,
+                                     float eps, int B, int H, int L, int d, int block_k, void* Q_out,
+                                     void* K_out, float* kbar, float* vbar, void* kbar_lp, void* vbar_lp,
+                                     void* stream);
+
 /* Bytes of device workspace sol_attn_fwd needs for this problem. The workspace holds the
  * persistent scheduler's work counter, the per-(b,h) kept-block counters and the sticky device
  * error word (a header of 4 * (4 + B*H) bytes rounded up to 256), followed by the keep bits of the

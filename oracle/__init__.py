@@ -15,3 +15,4 @@ from .sol_attn_oracle import (  # noqa: F401
     unit_forward,
     unit_terms,
 )
+from .qknorm_rope_oracle import qknorm_rope_pool_head, rms_norm, rope  # noqa: F401

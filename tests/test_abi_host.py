@@ -98,6 +98,28 @@ def test_pool_rejects_invalid_arguments(lib):
     assert lib.sol_attn_pool(p[0], p[1], sa.SOL_BF16, 1, 1, 0, 64, 128, p[2], p[3], p[4], p[5], None) == sa.SOL_EINVAL
 
 
+def rope_pool(lib, eps=1e-6, d=128, blk=128, B=1, H=2, L=1000, ptrs=None):
+    p = list(ptrs or P) + [ctypes.c_void_p(0x20000), ctypes.c_void_p(0x30000)]
+    return lib.sol_attn_qknorm_rope_pool(p[0], p[1], p[2], p[3], p[4], p[5], p[6], ctypes.c_float(eps), B, H, L, d, blk,
+                                         p[7], p[8], p[9], p[10], p[11], p[12], None)
+
+
+def test_qknorm_rope_pool_rejects_invalid_arguments(lib):
+    assert rope_pool(lib, eps=0.0) == sa.SOL_EINVAL
+    assert rope_pool(lib, eps=-1.0) == sa.SOL_EINVAL
+    assert rope_pool(lib, eps=math.inf) == sa.SOL_EINVAL
+    assert rope_pool(lib, L=0) == sa.SOL_EINVAL
+    nulls = list(P)
+    nulls[5] = None
+    assert rope_pool(lib, ptrs=nulls) == sa.SOL_EINVAL
+    misaligned = list(P)
+    misaligned[3] = ctypes.c_void_p(0x1004)
+    assert rope_pool(lib, ptrs=misaligned) == sa.SOL_EINVAL
+    assert rope_pool(lib, d=96) == sa.SOL_EUNSUPPORTED
+    assert rope_pool(lib, blk=8192) == sa.SOL_EUNSUPPORTED
+    assert rope_pool(lib, B=300, H=300) == sa.SOL_EUNSUPPORTED
+
+
 def test_check_device_error_rejects_null(lib):
     assert lib.sol_attn_check_device_error(None, None) == sa.SOL_EINVAL
 
