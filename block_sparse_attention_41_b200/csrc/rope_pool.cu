@@ -23,6 +23,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+constexpr int kBlocksPerCta = 4;  // consecutive key blocks per CTA: amortises launch and the final reduction
 
 struct RopePoolParams {
   const __nv_bfloat16* Q;
@@ -90,63 +91,67 @@ __global__ void __launch_bounds__(kThreads) sol_qknorm_rope_pool_kernel(const __
   __shared__ float s_part[2][RG][D];  // per row group partial sums of the stored keys / the values
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int jb = blockIdx.x, bh = blockIdx.y;
-  const int row0 = jb * p.block;
-  const int n = min(p.block, p.L - row0);
+  const int bh = blockIdx.y;
   const int cl = lane % LPR, sub = lane / LPR;
   const int c0 = cl * 8;
   const int rg = warp * RPW + sub;
   const float inv_d = 1.0f / static_cast<float>(D);
-  const size_t base = (static_cast<size_t>(bh) * p.L + row0) * D + c0;
+  const int jb_end = min(p.nkb, (static_cast<int>(blockIdx.x) + 1) * kBlocksPerCta);
+  for (int jb = blockIdx.x * kBlocksPerCta; jb < jb_end; ++jb) {
+    const int row0 = jb * p.block;
+    const int n = min(p.block, p.L - row0);
+    const size_t base = (static_cast<size_t>(bh) * p.L + row0) * D + c0;
 
-  float ak[8], av[8];
+    float ak[8], av[8];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) ak[k] = av[k] = 0.f;
-  // the loop runs the same number of times in every lane of a warp (the norm's shuffles need the
-  // whole warp); lanes past the block's last row carry zeros and store nothing
-  for (int rbase = warp * RPW; rbase < n; rbase += RG) {
-    const int r = rbase + sub;
-    const bool valid = r < n;
-    const size_t off = base + static_cast<size_t>(valid ? r : 0) * D;
-    const int t = row0 + (valid ? r : 0);
-    const float* cs = p.cs + static_cast<size_t>(t) * (D / 2);
-    const float* sn = p.sn + static_cast<size_t>(t) * (D / 2);
-    float xq[8], xk[8], xv[8];
-    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-    unpack8(valid ? __ldg(reinterpret_cast<const uint4*>(p.Q + off)) : zero, xq);
-    unpack8(valid ? __ldg(reinterpret_cast<const uint4*>(p.K + off)) : zero, xk);
-    unpack8(valid ? __ldg(reinterpret_cast<const uint4*>(p.V + off)) : zero, xv);
-    norm_rope_chunk<LPR>(xq, p.gq, cs, sn, c0, inv_d, p.eps, valid ? p.Qo + off : nullptr);
-    norm_rope_chunk<LPR>(xk, p.gk, cs, sn, c0, inv_d, p.eps, valid ? p.Ko + off : nullptr);
-    if (valid) {
+    for (int k = 0; k < 8; ++k) ak[k] = av[k] = 0.f;
+    // the loop runs the same number of times in every lane of a warp (the norm's shuffles need the
+    // whole warp); lanes past the block's last row carry zeros and store nothing
+    for (int rbase = warp * RPW; rbase < n; rbase += RG) {
+      const int r = rbase + sub;
+      const bool valid = r < n;
+      const size_t off = base + static_cast<size_t>(valid ? r : 0) * D;
+      const int t = row0 + (valid ? r : 0);
+      const float* cs = p.cs + static_cast<size_t>(t) * (D / 2);
+      const float* sn = p.sn + static_cast<size_t>(t) * (D / 2);
+      float xq[8], xk[8], xv[8];
+      const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+      unpack8(valid ? __ldg(reinterpret_cast<const uint4*>(p.Q + off)) : zero, xq);
+      unpack8(valid ? __ldg(reinterpret_cast<const uint4*>(p.K + off)) : zero, xk);
+      unpack8(valid ? __ldg(reinterpret_cast<const uint4*>(p.V + off)) : zero, xv);
+      norm_rope_chunk<LPR>(xq, p.gq, cs, sn, c0, inv_d, p.eps, valid ? p.Qo + off : nullptr);
+      norm_rope_chunk<LPR>(xk, p.gk, cs, sn, c0, inv_d, p.eps, valid ? p.Ko + off : nullptr);
+      if (valid) {
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        ak[k] += xk[k];
-        av[k] += xv[k];
+        for (int k = 0; k < 8; ++k) {
+          ak[k] += xk[k];
+          av[k] += xv[k];
+        }
       }
     }
-  }
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    s_part[0][rg][c0 + k] = ak[k];
-    s_part[1][rg][c0 + k] = av[k];
-  }
-  __syncthreads();
-  // thread t < 2 D: column t % D of the keys (t < D) or the values
-  if (tid < 2 * D) {
-    const int which = tid / D, c = tid % D;
-    float sum = 0.f;
-#pragma unroll 4
-    for (int k = 0; k < RG; ++k) sum += s_part[which][k][c];
-    const float mean = sum / static_cast<float>(n);
-    const size_t o = (static_cast<size_t>(bh) * p.nkb + jb) * D + c;
-    if (which == 0) {
-      p.kbar[o] = mean;
-      p.kbar_lp[o] = __float2bfloat16_rn(mean);
-    } else {
-      p.vbar[o] = mean;
-      p.vbar_lp[o] = __float2bfloat16_rn(mean);
+    for (int k = 0; k < 8; ++k) {
+      s_part[0][rg][c0 + k] = ak[k];
+      s_part[1][rg][c0 + k] = av[k];
     }
+    __syncthreads();
+    // thread t < 2 D: column t % D of the keys (t < D) or the values
+    if (tid < 2 * D) {
+      const int which = tid / D, c = tid % D;
+      float sum = 0.f;
+#pragma unroll 4
+      for (int k = 0; k < RG; ++k) sum += s_part[which][k][c];
+      const float mean = sum / static_cast<float>(n);
+      const size_t o = (static_cast<size_t>(bh) * p.nkb + jb) * D + c;
+      if (which == 0) {
+        p.kbar[o] = mean;
+        p.kbar_lp[o] = __float2bfloat16_rn(mean);
+      } else {
+        p.vbar[o] = mean;
+        p.vbar_lp[o] = __float2bfloat16_rn(mean);
+      }
+    }
+    __syncthreads();  // s_part is reused by the next block
   }
 }
 
@@ -170,7 +175,7 @@ cudaError_t launch_t(const RopePoolArgs& a, cudaStream_t stream) {
   p.block = a.block;
   p.nkb = (a.L + a.block - 1) / a.block;
   p.eps = a.eps;
-  const dim3 grid(p.nkb, a.BH);
+  const dim3 grid((p.nkb + kBlocksPerCta - 1) / kBlocksPerCta, a.BH);
   sol_qknorm_rope_pool_kernel<D><<<grid, kThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
