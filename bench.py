@@ -74,12 +74,23 @@ def reduce_max_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
+def code_tokens(src: str) -> str:
+    """C++/CUDA source without its comments and with whitespace runs collapsed: what the compiler
+    sees, so an edit to a comment does not read as a kernel change. String literals are kept whole."""
+    import re
+    tok = re.compile(r'"(?:\\.|[^"\\\n])*"|//[^\n]*|/\*.*?\*/', re.S)
+    src = tok.sub(lambda m: m.group(0) if m.group(0).startswith('"') else " ", src)
+    lines = (" ".join(ln.split()) for ln in src.splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def kernel_source_hash() -> str:
-    """First 16 hex digits of the sha256 of the tensor-core kernel's sources (as in profiles/)."""
+    """First 16 hex digits of the sha256 of the tensor-core kernel's code (its sources without
+    comments, see code_tokens), as recorded in the ncu summary under profiles/."""
     import hashlib
     csrc = os.path.join(ROOT, "block_sparse_attention_41_b200", "csrc")
-    data = b"".join(open(os.path.join(csrc, f), "rb").read() for f in ("fwd_tc.cu", "device_common.cuh"))
-    return hashlib.sha256(data).hexdigest()[:16]
+    data = "".join(code_tokens(open(os.path.join(csrc, f)).read()) for f in ("fwd_tc.cu", "device_common.cuh"))
+    return hashlib.sha256(data.encode()).hexdigest()[:16]
 
 
 def captured_traffic(w, key):

@@ -2,9 +2,13 @@
 //
 // The method (Sol-Attn project page, Abstract) in one kernel, per work unit = one 128-row
 // query block of one head:
-//   1. route    : q_bar from the Q tile in shared memory, proxy scores s_bar_j = q_bar.k_bar_j/sqrt(d)
-//                 against the fp32 pooled keys, threshold max - tau. The scores live only in shared
-//                 memory. The outputs are a kept-block list and a bitmask.
+//   1. route    : the unit's keep bits (one per key block), expanded into a kept-block list and a
+//                 pooled-tile list. They come either from the routing pass (route.cu: one read of
+//                 the pooled keys for several query blocks) or, when no bits are given, from this
+//                 kernel itself: q_bar from the Q tile in shared memory, proxy scores
+//                 s_bar_j = q_bar.k_bar_j/sqrt(d) against the fp32 pooled keys, threshold max - tau,
+//                 with the scores kept only in shared memory and the bitmask written out. Both ways
+//                 take the same fp32 operations in the same order, so they keep the same blocks.
 //   2. exact    : for each kept block, S = Q K^T (tcgen05, fp32 in TMEM), online softmax on CUDA cores,
 //                 P (bf16) written to TMEM, O += P V (tcgen05, A operand read from TMEM).
 //   3. correct  : every 128 consecutive pooled blocks that contain at least one skipped block form a

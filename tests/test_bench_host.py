@@ -63,3 +63,24 @@ def test_reference_arm_other_ranks_exit_quietly():
     r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "small_dit_L8192"],
                        cwd=ROOT, capture_output=True, text=True, timeout=300, env=env)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_kernel_code_hash_ignores_comments_but_not_code():
+    sys.path.insert(0, ROOT)
+    import bench
+    base = 'int a = 1;  // note\n/* block\n comment */\nconst char* s = "x // y";\n'
+    assert bench.code_tokens(base) == bench.code_tokens(base.replace("note", "other note") + "\n// more\n")
+    assert bench.code_tokens(base) != bench.code_tokens(base.replace("a = 1", "a = 2"))
+    assert '"x // y"' in bench.code_tokens(base)  # a string literal is code, not a comment
+
+
+def test_captured_traffic_is_dropped_once_the_kernel_code_changes(monkeypatch):
+    # the ncu summary's DRAM traffic is reported only while the kernel code is the captured one
+    sys.path.insert(0, ROOT)
+    import bench
+    from block_sparse_attention_41_b200 import workloads as wl
+    w = wl.WORKLOADS["video720p_L75600"]
+    got = bench.captured_traffic(w, "0.2")
+    assert got is None or got > 0
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0000000000000000")
+    assert bench.captured_traffic(w, "0.2") is None
