@@ -369,3 +369,242 @@ sol_status sol_attn_check_device_error(void* workspace, void* stream) {
 }
 
 }  // extern "C"
+
+// ---- host-buffer entry point: head chunks pipelined through caller-provided device scratch ------
+namespace {
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Where each buffer of sol_attn_fwd_host lives inside the scratch (byte offsets from its base).
+// Two slots of Q, K, V and O chunks, so that a chunk's upload, the previous chunk's compute and
+// the one before's download run at once. One set of pooled vectors and one workspace: the
+// compute of consecutive chunks is ordered on one stream.
+struct HostPlan {
+  int c = 0;                 // heads per chunk
+  size_t chunk_bytes = 0;    // one chunk of Q, K, V or O: c * L * d * element size
+  size_t in[2][3] = {};      // Q, K, V of slot 0 and 1
+  size_t out[2] = {};        // O of slot 0 and 1
+  size_t kbar = 0, vbar = 0, kbar_lp = 0, vbar_lp = 0;
+  size_t ws = 0, ws_bytes = 0;
+  size_t dens = 0;           // float32 [B * H]
+  size_t total = 0;
+};
+
+HostPlan host_plan(bool bf16, int B, int H, int L, int d, int block, int heads_per_chunk) {
+  HostPlan p;
+  p.c = heads_per_chunk < H ? heads_per_chunk : H;
+  const size_t es = bf16 ? 2 : 4;
+  const size_t nkb = (static_cast<size_t>(L) + block - 1) / block;
+  p.chunk_bytes = static_cast<size_t>(p.c) * L * d * es;
+  const size_t slot = round256(p.chunk_bytes);
+  size_t off = 0;
+  for (int s = 0; s < 2; ++s) {
+    for (int t = 0; t < 3; ++t) {
+      p.in[s][t] = off;
+      off += slot;
+    }
+    p.out[s] = off;
+    off += slot;
+  }
+  const size_t pooled_f32 = round256(static_cast<size_t>(p.c) * nkb * d * 4);
+  const size_t pooled_lp = bf16 ? round256(static_cast<size_t>(p.c) * nkb * d * 2) : 0;
+  p.kbar = off;
+  off += pooled_f32;
+  p.vbar = off;
+  off += pooled_f32;
+  p.kbar_lp = off;
+  off += pooled_lp;
+  p.vbar_lp = off;
+  off += pooled_lp;
+  p.ws = off;
+  p.ws_bytes = round256(ws_header_bytes(1, p.c) + ws_bits_bytes(1, p.c, L, block));
+  off += p.ws_bytes;
+  p.dens = off;
+  off += round256(static_cast<size_t>(B) * H * 4);
+  p.total = off;
+  return p;
+}
+
+// The checks of sol_attn_fwd that depend only on sizes, made once for the whole call so that a
+// bad argument is reported before any chunk is uploaded.
+sol_status host_validate(const void* Q, const void* K, const void* V, void* O, const float* tau, sol_dtype dt, int B,
+                         int H, int L, int d, int block, int n_force, int heads_per_chunk, const void* scratch) {
+  if (dt != SOL_F32 && dt != SOL_BF16) return fail(SOL_EINVAL, "unknown dtype %d", static_cast<int>(dt));
+  if (!size_ok(B, 1 << 16) || !size_ok(H, 1 << 16) || !size_ok(L, 1 << 28) || !size_ok(d, 1 << 16) ||
+      !size_ok(block, 1 << 20))
+    return fail(SOL_EINVAL, "sizes must be positive (B=%d H=%d L=%d d=%d block=%d)", B, H, L, d, block);
+  if (heads_per_chunk < 1) return fail(SOL_EINVAL, "heads_per_chunk=%d must be >= 1", heads_per_chunk);
+  if (Q == nullptr || K == nullptr || V == nullptr || O == nullptr || tau == nullptr || scratch == nullptr)
+    return fail(SOL_EINVAL, "Q, K, V, O, tau and scratch must be non-null");
+  if ((reinterpret_cast<uintptr_t>(scratch) & 255u) != 0) return fail(SOL_EINVAL, "scratch must be 256-byte aligned");
+  for (int h = 0; h < H; ++h)
+    if (std::isnan(tau[h]) || tau[h] < 0.f) return fail(SOL_EINVAL, "tau[%d]=%g must be >= 0 and not NaN", h, tau[h]);
+  if (dt == SOL_BF16) {
+    if (block != 128 || (d != 64 && d != 128))
+      return fail(SOL_EUNSUPPORTED, "bf16 path needs block 128 and d in {64, 128} (block=%d d=%d)", block, d);
+  } else {
+    if ((block != 32 && block != 64 && block != 128) || (d != 32 && d != 64 && d != 128))
+      return fail(SOL_EUNSUPPORTED, "fp32 path needs block in {32,64,128} and d in {32,64,128} (block=%d d=%d)",
+                  block, d);
+  }
+  const long long nkb = (static_cast<long long>(L) + block - 1) / block;
+  if (nkb > sol::kMaxKeyBlocks) return fail(SOL_EUNSUPPORTED, "N_kb=%lld exceeds %d", nkb, sol::kMaxKeyBlocks);
+  if (n_force < 0 || n_force > nkb) return fail(SOL_EINVAL, "n_force=%d must be in [0, N_kb=%lld]", n_force, nkb);
+  const int c = heads_per_chunk < H ? heads_per_chunk : H;
+  if (c > sol::kMaxHeads) return fail(SOL_EUNSUPPORTED, "heads_per_chunk=%d exceeds %d", c, sol::kMaxHeads);
+  if (static_cast<long long>(c) * nkb >= (1ll << 31)) return fail(SOL_EUNSUPPORTED, "chunk too large");
+  return SOL_OK;
+}
+
+// Q, K, V, O must not be device memory; the scratch must be device memory of the current device.
+sol_status host_check_memory(const void* const* host_ptrs, int n, const void* scratch) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  for (int i = 0; i < n; ++i) {
+    cudaPointerAttributes at;
+    e = cudaPointerGetAttributes(&at, host_ptrs[i]);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaPointerGetAttributes");
+    if (at.type == cudaMemoryTypeDevice) return fail(SOL_EINVAL, "Q, K, V and O must be host memory");
+  }
+  cudaPointerAttributes at;
+  e = cudaPointerGetAttributes(&at, scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaPointerGetAttributes");
+  if (at.type != cudaMemoryTypeDevice || at.device != dev)
+    return fail(SOL_EINVAL, "scratch must be device memory of the current device");
+  return SOL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sol_attn_fwd_host_scratch_bytes(sol_dtype dt, int B, int H, int L, int d, int block, int heads_per_chunk) {
+  if ((dt != SOL_F32 && dt != SOL_BF16) || B < 1 || H < 1 || L < 1 || d < 1 || block < 1 || heads_per_chunk < 1)
+    return 0;
+  return host_plan(dt == SOL_BF16, B, H, L, d, block, heads_per_chunk).total;
+}
+
+sol_status sol_attn_fwd_host(const void* Q, const void* K, const void* V, void* O, const float* tau, sol_dtype dt,
+                             int B, int H, int L, int d, int block, int n_force, int heads_per_chunk, float* density,
+                             void* scratch, size_t scratch_bytes, void* stream) {
+  g_last_error.clear();
+  sol_status st = host_validate(Q, K, V, O, tau, dt, B, H, L, d, block, n_force, heads_per_chunk, scratch);
+  if (st != SOL_OK) return st;
+  const bool bf16 = dt == SOL_BF16;
+  const HostPlan pl = host_plan(bf16, B, H, L, d, block, heads_per_chunk);
+  if (scratch_bytes < pl.total) return fail(SOL_EINVAL, "scratch too small (%zu < %zu bytes)", scratch_bytes, pl.total);
+  const void* host_ptrs[4] = {Q, K, V, O};
+  if ((st = host_check_memory(host_ptrs, 4, scratch)) != SOL_OK) return st;
+  int sms = 0;
+  if ((st = current_device(&sms)) != SOL_OK) return st;
+
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  constexpr int kEvents = 7;  // start, uploaded[2], computed[2], downloaded[2]
+  cudaEvent_t ev[kEvents] = {};
+  cudaEvent_t& ev_start = ev[0];
+  cudaEvent_t* ev_in = &ev[1];
+  cudaEvent_t* ev_comp = &ev[3];
+  cudaEvent_t* ev_out = &ev[5];
+  cudaError_t e = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking);
+  for (int i = 0; i < kEvents && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
+  if (e != cudaSuccess) st = cuda_fail(e, "stream / event creation");
+
+  // a clean workspace (its sticky error word too), then both copy streams start after `stream`'s
+  // earlier work, so a previous call on the same scratch has finished with it
+  if (st == SOL_OK && (e = cudaMemsetAsync(base + pl.ws, 0, pl.ws_bytes, s)) != cudaSuccess)
+    st = cuda_fail(e, "cudaMemsetAsync(workspace)");
+  if (st == SOL_OK && ((e = cudaEventRecord(ev_start, s)) != cudaSuccess ||
+                       (e = cudaStreamWaitEvent(s_in, ev_start, 0)) != cudaSuccess ||
+                       (e = cudaStreamWaitEvent(s_out, ev_start, 0)) != cudaSuccess))
+    st = cuda_fail(e, "stream ordering");
+
+  const uint8_t* hq = static_cast<const uint8_t*>(Q);
+  const uint8_t* hk = static_cast<const uint8_t*>(K);
+  const uint8_t* hv = static_cast<const uint8_t*>(V);
+  uint8_t* ho = static_cast<uint8_t*>(O);
+  const size_t head_bytes = static_cast<size_t>(L) * d * (bf16 ? 2 : 4);
+  float* dens_dev = reinterpret_cast<float*>(base + pl.dens);
+  int chunk = 0;
+  for (int b = 0; b < B && st == SOL_OK; ++b) {
+    for (int h0 = 0; h0 < H && st == SOL_OK; h0 += pl.c, ++chunk) {
+      const int ce = (H - h0) < pl.c ? (H - h0) : pl.c;
+      const int sl = chunk & 1;
+      const size_t host_off = (static_cast<size_t>(b) * H + h0) * head_bytes;
+      const size_t bytes = static_cast<size_t>(ce) * head_bytes;  // <= pl.chunk_bytes
+      uint8_t* dq = base + pl.in[sl][0];
+      uint8_t* dk = base + pl.in[sl][1];
+      uint8_t* dv = base + pl.in[sl][2];
+      uint8_t* dout = base + pl.out[sl];
+      // upload: the slot's inputs are free once the compute of chunk - 2 has finished
+      if (chunk >= 2 && (e = cudaStreamWaitEvent(s_in, ev_comp[sl], 0)) != cudaSuccess) {
+        st = cuda_fail(e, "stream ordering");
+        break;
+      }
+      if ((e = cudaMemcpyAsync(dq, hq + host_off, bytes, cudaMemcpyHostToDevice, s_in)) != cudaSuccess ||
+          (e = cudaMemcpyAsync(dk, hk + host_off, bytes, cudaMemcpyHostToDevice, s_in)) != cudaSuccess ||
+          (e = cudaMemcpyAsync(dv, hv + host_off, bytes, cudaMemcpyHostToDevice, s_in)) != cudaSuccess ||
+          (e = cudaEventRecord(ev_in[sl], s_in)) != cudaSuccess) {
+        st = cuda_fail(e, "upload");
+        break;
+      }
+      // compute: after this chunk's upload, and after the download of chunk - 2 freed the O slot
+      if ((e = cudaStreamWaitEvent(s, ev_in[sl], 0)) != cudaSuccess ||
+          (chunk >= 2 && (e = cudaStreamWaitEvent(s, ev_out[sl], 0)) != cudaSuccess)) {
+        st = cuda_fail(e, "stream ordering");
+        break;
+      }
+      float* kbar = reinterpret_cast<float*>(base + pl.kbar);
+      float* vbar = reinterpret_cast<float*>(base + pl.vbar);
+      void* klp = bf16 ? static_cast<void*>(base + pl.kbar_lp) : nullptr;
+      void* vlp = bf16 ? static_cast<void*>(base + pl.vbar_lp) : nullptr;
+      st = sol_attn_pool(dk, dv, dt, 1, ce, L, d, block, kbar, vbar, klp, vlp, stream);
+      if (st != SOL_OK) break;
+      st = sol_attn_fwd(dq, dk, dv, kbar, vbar, klp, vlp, tau + h0, dt, 1, ce, L, d, block, block, n_force, dout,
+                        nullptr, density != nullptr ? dens_dev + static_cast<size_t>(b) * H + h0 : nullptr,
+                        base + pl.ws, pl.ws_bytes, stream);
+      if (st != SOL_OK) break;
+      if ((e = cudaEventRecord(ev_comp[sl], s)) != cudaSuccess) {
+        st = cuda_fail(e, "stream ordering");
+        break;
+      }
+      // download
+      if ((e = cudaStreamWaitEvent(s_out, ev_comp[sl], 0)) != cudaSuccess ||
+          (e = cudaMemcpyAsync(ho + host_off, dout, bytes, cudaMemcpyDeviceToHost, s_out)) != cudaSuccess ||
+          (e = cudaEventRecord(ev_out[sl], s_out)) != cudaSuccess) {
+        st = cuda_fail(e, "download");
+        break;
+      }
+    }
+  }
+  if (st == SOL_OK && density != nullptr &&
+      (e = cudaMemcpyAsync(density, dens_dev, static_cast<size_t>(B) * H * 4, cudaMemcpyDeviceToHost, s)) !=
+          cudaSuccess)
+    st = cuda_fail(e, "density download");
+
+  // whatever happened above, nothing may still be copying into the caller's buffers on return
+  cudaError_t es = cudaSuccess;
+  if (s_in != nullptr && (e = cudaStreamSynchronize(s_in)) != cudaSuccess) es = e;
+  if (s_out != nullptr && (e = cudaStreamSynchronize(s_out)) != cudaSuccess) es = e;
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) es = e;
+  for (int i = 0; i < kEvents; ++i)
+    if (ev[i] != nullptr) cudaEventDestroy(ev[i]);
+  if (s_in != nullptr) cudaStreamDestroy(s_in);
+  if (s_out != nullptr) cudaStreamDestroy(s_out);
+  if (st != SOL_OK) return st;  // its reason is already in the last-error string
+  if (es != cudaSuccess) return cuda_fail(es, "cudaStreamSynchronize");
+  uint32_t words[2] = {0, 0};
+  if ((e = cudaMemcpy(words, base + pl.ws, sizeof(words), cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e, "cudaMemcpy(error word)");
+  if (words[0] != 0) {
+    static const char* roles[] = {"?", "producer", "mma", "softmax", "router"};
+    return fail(SOL_ETIMEOUT, "device wait expired (first in the %s role); the outputs are incomplete",
+                roles[words[1] < 5 ? words[1] : 0]);
+  }
+  return SOL_OK;
+}
+
+}  // extern "C"

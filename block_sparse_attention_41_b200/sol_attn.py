@@ -31,6 +31,8 @@ EXPORTED = (
     "sol_attn_debug_drop_one_load",
     "sol_attn_fwd_noalloc",
     "sol_attn_qknorm_rope_pool",
+    "sol_attn_fwd_host_scratch_bytes",
+    "sol_attn_fwd_host",
 )
 
 
@@ -73,6 +75,11 @@ def load_library() -> ctypes.CDLL:
     lib.sol_attn_qknorm_rope_pool.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, i32, i32, i32, i32,
                                               vp, vp, vp, vp, vp, vp, vp]
     lib.sol_attn_qknorm_rope_pool.restype = i32
+    lib.sol_attn_fwd_host_scratch_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32]
+    lib.sol_attn_fwd_host_scratch_bytes.restype = ctypes.c_size_t
+    lib.sol_attn_fwd_host.argtypes = [vp, vp, vp, vp, f32p, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp,
+                                      ctypes.c_size_t, vp]
+    lib.sol_attn_fwd_host.restype = i32
     lib.sol_attn_check_device_error.argtypes = [vp, vp]
     lib.sol_attn_check_device_error.restype = i32
     lib.sol_attn_debug_drop_one_load.argtypes = [i32]
@@ -263,6 +270,57 @@ def sol_attn(Q, K, V, tau, block: int = 128, n_force: int = 0, want_mask: bool =
     O = sol_attn_fwd(Q, K, V, kbar, vbar, kbar_lp, vbar_lp, tau, block, block, n_force, kept_mask=mask,
                      density=dens, workspace=workspace, stream=stream)
     return O, mask, dens
+
+
+def sol_attn_fwd_host_scratch_bytes(dtype: torch.dtype, B: int, H: int, L: int, d: int, block: int,
+                                    heads_per_chunk: int) -> int:
+    code = SOL_BF16 if dtype == torch.bfloat16 else SOL_F32 if dtype == torch.float32 else -1
+    return int(load_library().sol_attn_fwd_host_scratch_bytes(code, B, H, L, d, block, heads_per_chunk))
+
+
+def default_heads_per_chunk(H: int) -> int:
+    """About 20 chunks per batch entry: the pipeline fills after one small upload."""
+    return max(1, -(-H // 20))
+
+
+def sol_attn_fwd_host(Q, K, V, tau, block: int = 128, n_force: int = 0, heads_per_chunk: Optional[int] = None,
+                      O=None, want_density: bool = False, scratch=None, stream=None):
+    """The whole path (pool + forward) on HOST tensors, pipelined by head chunks through device
+    scratch. Synchronous: returns (O, density or None) with both in host memory.
+
+    Q, K, V: CPU tensors [B, H, L, d] (pinned for copy/compute overlap). `scratch`: a CUDA uint8
+    tensor of at least sol_attn_fwd_host_scratch_bytes(...) bytes on the current device.
+    """
+    for n, t in (("Q", Q), ("K", K), ("V", V)):
+        if not isinstance(t, torch.Tensor) or t.device.type != "cpu":
+            raise TypeError(f"{n} must be a CPU tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+        if t.dtype != Q.dtype or t.shape != Q.shape:
+            raise ValueError("Q, K and V must have the same dtype and shape [B, H, L, d]")
+    B, H, L, d = Q.shape
+    dt = _dtype_code(Q)
+    tau = [float(x) for x in tau]
+    if len(tau) != H:
+        raise ValueError(f"tau must hold H={H} values")
+    c = default_heads_per_chunk(H) if heads_per_chunk is None else int(heads_per_chunk)
+    pinned = Q.is_pinned()
+    if O is None:
+        O = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=pinned)
+    elif O.device.type != "cpu" or not O.is_contiguous() or O.dtype != Q.dtype or O.shape != Q.shape:
+        raise ValueError("O must be a contiguous CPU tensor of Q's dtype and shape")
+    dens = torch.empty((B, H), dtype=torch.float32, pin_memory=pinned) if want_density else None
+    if scratch is None:
+        scratch = torch.empty(sol_attn_fwd_host_scratch_bytes(Q.dtype, B, H, L, d, block, c), dtype=torch.uint8,
+                              device=torch.device("cuda", torch.cuda.current_device()))
+    else:
+        _need_cuda("scratch", scratch, torch.uint8)
+    tau_c = (ctypes.c_float * H)(*tau)
+    st = load_library().sol_attn_fwd_host(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(O), tau_c, dt, B, H, L, d, block, int(n_force), c, _ptr(dens),
+        _ptr(scratch), scratch.numel(), _stream(stream))
+    _check(st, "sol_attn_fwd_host")
+    return O, dens
 
 
 def tau_list(values) -> list:

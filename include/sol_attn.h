@@ -26,7 +26,8 @@
  *     caller; the library allocates nothing and keeps no global state (the one exception is the
  *     static device array of sol_attn_fwd_noalloc, described there).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). Every call
- *     that launches work is asynchronous on that stream.
+ *     that launches work is asynchronous on that stream, except sol_attn_fwd_host, whose host
+ *     buffers make it synchronous (described there).
  *   - Arguments are validated on the host before any launch. Invalid ones return SOL_EINVAL,
  *     and shapes or dtypes the kernels do not implement return SOL_EUNSUPPORTED. In both cases
  *     nothing is launched. A failed CUDA runtime call returns SOL_ECUDA.
@@ -179,6 +180,47 @@ sol_status sol_attn_fwd_noalloc(const void* Q, const void* K, const void* V, con
                                 const float* tau, sol_dtype dt, int B, int H, int L, int d,
                                 int block_q, int block_k, int n_force, void* O, uint8_t* kept_mask,
                                 float* density, void* stream);
+
+/* Bytes of device scratch sol_attn_fwd_host needs (0 for invalid sizes or dtype). The scratch holds
+ * two slots of Q, K, V and O for `heads_per_chunk` heads, one set of pooled vectors for that many
+ * heads, one workspace and B*H density words, each rounded up to 256 bytes. For bf16, H=40,
+ * L=75600, d=128 with 2 heads per chunk that is 0.31 GB. */
+size_t sol_attn_fwd_host_scratch_bytes(sol_dtype dt, int B, int H, int L, int d, int block,
+                                       int heads_per_chunk);
+
+/* The whole path (sol_attn_pool, then sol_attn_fwd) on inputs and output in HOST memory. This is
+ * the same operation, with the same kernels and results, for callers whose tensors live on the
+ * host. The pages describe no such call; it is a deployment convenience of this library.
+ *
+ * Heads are independent, so the call cuts each batch entry's H heads into chunks of
+ * `heads_per_chunk` and pipelines them through two slots of the device scratch. Chunk c is
+ * uploaded on one copy stream while chunk c-1 is pooled and attended on `stream`, and chunk c-2's
+ * output is downloaded on a second copy stream. With pinned host memory the uploads, the compute
+ * and the downloads overlap, so the call takes about as long as its slowest part (usually the
+ * upload of Q, K and V over the host link) plus one chunk. Pageable host memory gives the same
+ * results without that overlap. The copy streams and the events are created and destroyed inside
+ * the call.
+ *
+ *   Q, K, V    HOST, [B, H, L, d] in dtype `dt` (pinned for overlap; must not be device memory)
+ *   O          HOST, [B, H, L, d] in dtype `dt`: the output
+ *   tau        HOST, float32 [H], as for sol_attn_fwd
+ *   block      block_q = block_k; the sizes supported are those of sol_attn_fwd
+ *   n_force    as for sol_attn_fwd
+ *   heads_per_chunk  >= 1 (values above H mean H): smaller chunks start the pipeline sooner,
+ *              larger ones give each launch more work units
+ *   density    HOST, float32 [B, H] or NULL: kept blocks / (N_qb * N_kb) per head
+ *   scratch    device memory of the current device, 256-byte aligned, at least
+ *              sol_attn_fwd_host_scratch_bytes(...) bytes; no zeroing needed
+ *   stream     the compute stream. Work enqueued on it earlier finishes before the call's first
+ *              upload starts.
+ * Synchronous: it returns once O and density are in host memory, or after a failure, once
+ * nothing the call started is still running. All size checks run before the first copy. A
+ * bounded-wait expiry in any chunk returns SOL_ETIMEOUT, and the outputs are then incomplete.
+ * Not usable inside a CUDA graph capture. */
+sol_status sol_attn_fwd_host(const void* Q, const void* K, const void* V, void* O, const float* tau,
+                             sol_dtype dt, int B, int H, int L, int d, int block, int n_force,
+                             int heads_per_chunk, float* density, void* scratch, size_t scratch_bytes,
+                             void* stream);
 
 /* Test hook for the failure-detection path. mode 0 (default) = normal operation. mode 1 makes
  * the next sol_attn_fwd launch (SOL_BF16 path) skip one K-tile load, so the consumer's bounded

@@ -129,3 +129,55 @@ def test_binding_fails_loudly_without_cuda_tensors(lib):
     x = torch.zeros(1, 1, 8, 64)
     with pytest.raises(TypeError):
         sa.sol_attn_pool(x, x, 128)
+
+
+def test_host_entry_scratch_size(lib):
+    # two slots of Q, K, V, O for 2 heads, pooled fp32 + bf16 vectors for 2 heads, the workspace
+    # of a 2-head call and 40 density words, each rounded up to 256 bytes
+    r = lambda x: -(-x // 256) * 256  # noqa: E731
+    L, d, c, H, nkb = 75600, 128, 2, 40, 591
+    ws = r(r((4 + c) * 4) + r(c * nkb * 19 * 4))
+    want = 8 * r(c * L * d * 2) + 2 * r(c * nkb * d * 4) + 2 * r(c * nkb * d * 2) + ws + r(H * 4)
+    assert lib.sol_attn_fwd_host_scratch_bytes(sa.SOL_BF16, 1, H, L, d, 128, c) == want
+    # fp32: 4-byte elements, no bf16 mirrors
+    want32 = 8 * r(c * 1000 * 64 * 4) + 2 * r(c * 16 * 64 * 4) + r(r((4 + c) * 4) + r(c * 16 * 1 * 4)) + r(3 * 4)
+    assert lib.sol_attn_fwd_host_scratch_bytes(sa.SOL_F32, 1, 3, 1000, 64, 64, c) == want32
+    # more heads per chunk than heads: one chunk of H heads
+    assert (lib.sol_attn_fwd_host_scratch_bytes(sa.SOL_BF16, 2, 3, 1000, 64, 128, 99) ==
+            lib.sol_attn_fwd_host_scratch_bytes(sa.SOL_BF16, 2, 3, 1000, 64, 128, 3))
+    for bad in ((7, 1, 3, 1000, 64, 128, 1), (sa.SOL_BF16, 0, 3, 1000, 64, 128, 1),
+                (sa.SOL_BF16, 1, 3, 1000, 64, 128, 0)):
+        assert lib.sol_attn_fwd_host_scratch_bytes(*bad) == 0
+
+
+def fwd_host(lib, dt=sa.SOL_BF16, B=1, H=2, L=1000, d=128, blk=128, n_force=0, tau=(1.0, 1.0), chunk=1,
+             scratch=ctypes.c_void_p(0x100000), nbytes=1 << 40, o=P[3]):
+    tau_c = (ctypes.c_float * len(tau))(*tau)
+    return lib.sol_attn_fwd_host(P[0], P[1], P[2], o, tau_c, dt, B, H, L, d, blk, n_force, chunk, None, scratch,
+                                 nbytes, None)
+
+
+def test_host_entry_rejects_invalid_arguments_before_any_copy(lib):
+    assert fwd_host(lib, tau=(1.0, -1.0)) == sa.SOL_EINVAL
+    assert fwd_host(lib, chunk=0) == sa.SOL_EINVAL
+    assert "heads_per_chunk" in lib.sol_attn_last_error().decode()
+    assert fwd_host(lib, o=None) == sa.SOL_EINVAL
+    assert fwd_host(lib, scratch=ctypes.c_void_p(0x100010)) == sa.SOL_EINVAL  # not 256-byte aligned
+    assert fwd_host(lib, nbytes=4096) == sa.SOL_EINVAL
+    assert "scratch too small" in lib.sol_attn_last_error().decode()
+    assert fwd_host(lib, n_force=9) == sa.SOL_EINVAL
+    assert fwd_host(lib, d=96) == sa.SOL_EUNSUPPORTED
+    assert fwd_host(lib, dt=sa.SOL_F32, blk=48) == sa.SOL_EUNSUPPORTED
+    assert fwd_host(lib, L=4096 * 128 + 1) == sa.SOL_EUNSUPPORTED
+    # valid sizes: the next check asks the runtime where the pointers live, which fails without a
+    # GPU (SOL_ECUDA) and rejects the fake scratch address with one (SOL_EINVAL); no copy is made
+    assert fwd_host(lib) in (sa.SOL_ECUDA, sa.SOL_EINVAL)
+
+
+def test_host_binding_rejects_non_host_tensors(lib):
+    import torch
+    with pytest.raises(TypeError):
+        sa.sol_attn_fwd_host([1.0], [1.0], [1.0], [1.0])
+    x = torch.zeros(1, 1, 8, 64)
+    with pytest.raises(ValueError):
+        sa.sol_attn_fwd_host(x, x, torch.zeros(1, 1, 8, 32), [1.0])
