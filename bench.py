@@ -173,9 +173,11 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------------ CPU oracle
-def oracle_sample(w, tau, budget_s: float, max_units: int = 64, seed_offset: int = 77):
+def oracle_sample(w, tau, budget_s: float, max_units: int = 64, seed_offset: int = 77, collect=None):
     """Time the float64 oracle, as it stands, on seeded query-block units of the workload until
-    `budget_s` seconds of work are done. Returns (kept tiles processed, seconds, units, threads)."""
+    `budget_s` seconds of work are done. Returns (kept tiles processed, seconds, units, threads).
+    If `collect` is a list, each unit's (b, h, i, O rows, keep row) is appended to it, outside the
+    timed part."""
     import oracle
     try:
         from threadpoolctl import threadpool_info
@@ -190,9 +192,11 @@ def oracle_sample(w, tau, budget_s: float, max_units: int = 64, seed_offset: int
             heads = {(b, h): [x.astype(np.float64) for x in wl.head_tensors(w, b, h)]}
         q, k, v = heads[(b, h)]
         t0 = time.perf_counter()
-        _, keep, _, _ = oracle.forward_head(q, k, v, float(tau[h]), w.block, w.block, w.n_force, units=[i])
+        O_ref, keep, _, _ = oracle.forward_head(q, k, v, float(tau[h]), w.block, w.block, w.n_force, units=[i])
         elapsed += time.perf_counter() - t0
         kept_tiles += int(keep[i].sum())
+        if collect is not None:
+            collect.append((b, h, i, O_ref[i * w.block: (i + 1) * w.block], keep[i].copy()))
         done += 1
         if elapsed >= budget_s:
             break
@@ -252,6 +256,52 @@ def measure_qknorm_rope_pool(w, Q, K, V, stream, pk, cpu_ok, max_over_ranks, bar
         out["cpu_baseline"] = {"value": sample_bytes / secs / 1e9, "unit": "GB/s", "kind": "oracle",
                                "sample": f"{rows} tokens of one head ({secs:.2f} s of float64 oracle work)"}
     return out
+
+
+def per_run_report(w, Q, K, V, kbar, vbar, klp, vlp, tau, key, O, dens, ws, stream):
+    """One untimed call with the kept mask: per-head densities, kept-tile FLOPs over valid tokens
+    only (the partial last query and key blocks count their valid rows and columns), the
+    correction's algorithmic FLOPs (4 m_i d per skipped block), and the oracle's near-threshold
+    band count for these thresholds (from the calibration table)."""
+    import torch
+    from block_sparse_attention_41_b200 import sol_attn as sa
+    B, H, L, d, blk, nb = w.B, w.H, w.L, w.d, w.block, w.n_blocks
+    mask = torch.empty((B, H, nb, nb), dtype=torch.uint8, device=Q.device)
+    sa.sol_attn_fwd(Q, K, V, kbar, vbar, klp, vlp, tau, blk, blk, w.n_force, O=O, kept_mask=mask, density=dens,
+                    workspace=ws, stream=stream)
+    torch.cuda.synchronize()
+    sa.sol_attn_check_device_error(ws)
+    valid = torch.full((nb,), blk, dtype=torch.int64, device=Q.device)
+    valid[-1] = L - (nb - 1) * blk
+    mk = mask.to(torch.int64)
+    kept_valid = int((mk * (valid[:, None] * valid[None, :])).sum())
+    skipped_rows = int(((1 - mk) * valid[:, None]).sum())
+    with open(os.path.join(ROOT, "tests", "golden", "tau.json")) as f:
+        band = json.load(f)["workloads"][w.name][key].get("band_b0")
+    units = wl.sample_units(w, 64, seed_offset=77)
+    out = {"density_per_head": [round(float(x), 6) for x in dens.view(-1).tolist()],
+           "kept_flops_valid_tokens": 4.0 * d * kept_valid,
+           "correction_flops": 4.0 * d * skipped_rows,
+           "band_entries_oracle": int(sum(band)) if band is not None else None,
+           "_mask_rows": {(b, h, i): mask[b, h, i].cpu().numpy().astype(bool) for b, h, i in units}}
+    del mask, mk
+    return out
+
+
+def sample_parity(collected, gpu_rows, mask_rows):
+    """GPU output rows against the oracle's rows of the same units. A unit whose kept set differs
+    (a near-threshold entry that fp32 and float64 routing decide differently) is counted, not
+    compared: the tests compare those with the GPU's bits."""
+    errs, same = [], 0
+    for b, h, i, o_ref, keep in collected:
+        if not np.array_equal(keep, mask_rows[(b, h, i)]):
+            continue
+        same += 1
+        o_gpu = gpu_rows[(b, h, i)][: o_ref.shape[0]]
+        errs.append(np.abs(o_gpu - o_ref))
+    e = np.concatenate([x.ravel() for x in errs]) if errs else np.zeros(1)
+    return {"units": len(collected), "units_compared": same, "max_abs": float(e.max()), "mean_abs": float(e.mean()),
+            "tol_max_abs": 2e-2, "tol_mean_abs": 2e-3}
 
 
 def run_reference(args, w):
@@ -356,6 +406,7 @@ def run_ours(args, w):
     sa.sol_attn_check_device_error(ws)
     kept = int(round(float(dens.double().sum()) * nb * nb))
     flops = kept_tile_flops(kept, w)
+    per_run = per_run_report(w, Q, K, V, kbar, vbar, klp, vlp, tau, key, O, dens, ws, stream)
 
     for _ in range(args.warmup):
         step(tau)
@@ -373,6 +424,9 @@ def run_ours(args, w):
     barrier()
     torch.cuda.synchronize()
     sa.sol_attn_check_device_error(ws)
+    # the timed steps left the timed density's output in O: keep the rows of the oracle's sample units
+    cpu_units = wl.sample_units(w, 64, seed_offset=77) if rank == 0 and world == 1 and not args.no_cpu_baseline else []
+    gpu_rows = {(b, h, i): O[b, h, i * blk: (i + 1) * blk].double().cpu().numpy() for b, h, i in cpu_units}
     ms_total = max_over_ranks(t0.elapsed_time(t1))
     ms_step = ms_total / args.steps
     fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_ev)
@@ -445,11 +499,14 @@ def run_ours(args, w):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tiles, secs, units, threads = oracle_sample(w, tau, args.cpu_budget)
+        collected = []
+        tiles, secs, units, threads = oracle_sample(w, tau, args.cpu_budget, collect=collected)
         cpu = {"value": kept_tile_flops(tiles, w) / secs / 1e12, "unit": "TFLOP/s", "cores": threads,
                "kind": "oracle",
                "sample": f"{units} seeded query-block units of {w.name} at density {key} "
                          f"({secs:.1f} s of float64 oracle work, extrapolated per kept tile)"}
+        per_run["parity_sample"] = sample_parity(collected, gpu_rows, per_run.pop("_mask_rows"))
+    per_run.pop("_mask_rows", None)
 
     traffic = captured_traffic(w, key)
 
@@ -478,6 +535,7 @@ def run_ours(args, w):
             "clocks": clocks,
             "sweep": sweep,
             "next_rows": next_rows,
+            "per_run": per_run,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -84,3 +84,26 @@ def test_captured_traffic_is_dropped_once_the_kernel_code_changes(monkeypatch):
     assert got is None or got > 0
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0000000000000000")
     assert bench.captured_traffic(w, "0.2") is None
+
+
+def test_sampled_parity_report_compares_only_units_with_the_same_kept_set():
+    # the oracle's own sampled rows, collected outside its timed part, against themselves plus a
+    # known error; a unit whose mask row differs is counted but not compared
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import bench
+    from block_sparse_attention_41_b200 import workloads as wl
+    w = wl.WORKLOADS["small_dit_L8192"]
+    tau = bench.tau_for(w, bench.density_keys(w)[0])
+    got = []
+    _, _, n, _ = bench.oracle_sample(w, tau, budget_s=0.5, max_units=4, collect=got)
+    assert len(got) == n >= 1
+    b, h, i, rows, keep = got[0]
+    assert rows.shape == (w.block, w.d) and np.isfinite(rows).all() and keep.dtype == bool and keep.any()
+    gpu = {(b_, h_, i_): r + 1e-3 for b_, h_, i_, r, _ in got}
+    masks = {(b_, h_, i_): k.copy() for b_, h_, i_, _, k in got}
+    rep = bench.sample_parity(got, gpu, masks)
+    assert rep["units"] == n and rep["units_compared"] == n
+    assert abs(rep["max_abs"] - 1e-3) < 1e-12 and abs(rep["mean_abs"] - 1e-3) < 1e-12
+    masks[(b, h, i)] = ~masks[(b, h, i)]
+    assert bench.sample_parity(got, gpu, masks)["units_compared"] == n - 1
