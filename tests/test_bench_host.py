@@ -107,3 +107,16 @@ def test_sampled_parity_report_compares_only_units_with_the_same_kept_set():
     assert abs(rep["max_abs"] - 1e-3) < 1e-12 and abs(rep["mean_abs"] - 1e-3) < 1e-12
     masks[(b, h, i)] = ~masks[(b, h, i)]
     assert bench.sample_parity(got, gpu, masks)["units_compared"] == n - 1
+
+
+def test_cpu_sample_units_come_from_a_few_fixed_heads():
+    sys.path.insert(0, ROOT)
+    import bench
+    from block_sparse_attention_41_b200 import workloads as wl
+    w = wl.WORKLOADS["video720p_L75600"]
+    a = bench.cpu_sample_units(w, 192, 77)
+    assert a == bench.cpu_sample_units(w, 192, 77) and a == sorted(a) and len(set(a)) == 192
+    b = bench.cpu_sample_units(w, 192, 100)
+    heads = {(u[0], u[1]) for u in a}
+    assert len(heads) == bench.CPU_SAMPLE_HEADS and {(u[0], u[1]) for u in b} == heads and a != b
+    assert all(0 <= u[2] < w.n_blocks for u in a)
