@@ -16,3 +16,4 @@ from .sol_attn_oracle import (  # noqa: F401
     unit_terms,
 )
 from .qknorm_rope_oracle import qknorm_rope_pool_head, rms_norm, rope  # noqa: F401
+from .mxfp8_oracle import forward_head_mx, int8_quantize_tiles, mx_quantize, no_quantize, round_e4m3  # noqa: F401,E501
