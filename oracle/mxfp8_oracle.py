@@ -33,6 +33,10 @@ the plainest reading that a Blackwell block-scaled tensor-core kernel computes:
   met. The row sum is the sum of the quantized weights, the same values the PV product uses.
   O_r = sum_tiles Pq_tile Vq_tile / sum_tiles sum(Pq_tile).
 
+Parity with an upstream low-precision kernel is unpinned: the pages give no formula. The pins
+in tests/test_oracle_lowp_pins.py tie this oracle to the OCP formats' definitions and to the bf16
+definition.
+
 Every function takes and returns float64 arrays.
 """
 from __future__ import annotations

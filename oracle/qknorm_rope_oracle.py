@@ -20,6 +20,9 @@ this oracle takes the textbook forms:
   ``sol_attn_oracle.pool_blocks``), taken from the rotated keys after their rounding to the
   output dtype, so they equal what pooling the stored keys would give.
 
+Parity with upstream's fused kernel is unpinned: the pages give no formula. The pins in
+tests/test_oracle_rope_pins.py tie this oracle to the textbook forms above.
+
 Every function takes and returns float64 arrays.
 """
 from __future__ import annotations

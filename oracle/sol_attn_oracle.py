@@ -32,6 +32,10 @@ Readings taken where the pages are silent:
 * forced blocks are OR-ed in after routing. The max M_i runs over all blocks, forced ones
   included. Forced blocks count toward density.
 
+Parity with upstream Sol-Attn's own arithmetic is unpinned: the pages print no formula. The
+pins in tests/test_oracle_pins.py tie this oracle to the definition above, through dense special
+cases, invariants, brute force on tiny inputs and a hand-derived example.
+
 The softmax is the two-pass form (the exact row max first, then the weighted sums). It is
 deliberately not the online form used on the GPU. Every function takes float64 arrays.
 """
