@@ -45,7 +45,7 @@ def _oracle_attn(Q, K, V, tau, block, n_force):
     return torch.from_numpy(O)
 
 
-def _rank(rank, world, port, case, mismatch, out):
+def _rank(rank, world, port, case, mismatch, out, chunk=None):
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
@@ -55,10 +55,13 @@ def _rank(rank, world, port, case, mismatch, out):
         Q, K, V = (torch.from_numpy(x) for x in _inputs(B, H, L, d, seed))
         a = sum(lens[:rank])
         sl = slice(a, a + lens[rank])
-        Hr = H - 1 if mismatch and rank == 1 else H
+        Hr = H - 1 if mismatch == "heads" and rank == 1 else H
         q, k, v = (x[:, :Hr, sl].contiguous() for x in (Q, K, V))
+        if mismatch == "k_shape" and rank == 1:
+            k = k[:, :, : max(0, k.shape[2] - 1)].contiguous()
         try:
-            o = cp.sol_attn_context_parallel(q, k, v, tau[:Hr], block=blk, n_force=n_force, attn=_oracle_attn)
+            o = cp.sol_attn_context_parallel(q, k, v, tau[:Hr], block=blk, n_force=n_force, attn=_oracle_attn,
+                                             heads_per_chunk=chunk)
             out[rank] = o.numpy()
         except ValueError as e:
             out[rank] = f"ValueError: {e}"
@@ -66,10 +69,10 @@ def _rank(rank, world, port, case, mismatch, out):
         dist.destroy_process_group()
 
 
-def _run(world, case, mismatch=False):
+def _run(world, case, mismatch=None, chunk=None):
     mgr = mp.Manager()
     out = mgr.dict()
-    mp.spawn(_rank, args=(world, _free_port(), case, mismatch, out), nprocs=world, join=True)
+    mp.spawn(_rank, args=(world, _free_port(), case, mismatch, out, chunk), nprocs=world, join=True)
     return dict(out)
 
 
@@ -83,17 +86,20 @@ def test_head_groups_and_sequence_ranges():
     assert cp.seq_shard_ranges(100, 4, 64) == [(0, 64), (64, 100), (100, 100), (100, 100)]
 
 
-@pytest.mark.parametrize("world,H,lens,n_force", [
-    (2, 5, [300, 400], 0),
-    (3, 5, [128, 250, 322], 2),
-    (4, 3, [100, 0, 350, 250], 1),  # an empty token range, and a rank without a head
+@pytest.mark.parametrize("world,H,lens,n_force,chunk", [
+    (2, 5, [300, 400], 0, None),
+    (3, 5, [128, 250, 322], 2, None),
+    (4, 3, [100, 0, 350, 250], 1, None),  # an empty token range, and a rank without a head
+    (2, 5, [300, 400], 0, 1),             # groups of 3 and 2 heads in 3 pipelined chunks
+    (3, 5, [128, 250, 322], 1, 1),        # the third rank's group runs out after one chunk
+    (2, 5, [350, 350], 0, 2),             # chunks of 2 and 1 heads
 ])
-def test_context_parallel_equals_the_single_process_oracle(world, H, lens, n_force):
+def test_context_parallel_equals_the_single_process_oracle(world, H, lens, n_force, chunk):
     B, d, blk = 1, 16, 64
     L = sum(lens)
     tau = [0.0, 0.7, math.inf, 1.3, 0.2][:H]
     case = (B, H, L, d, blk, n_force, lens, tau, 17 + world)
-    got = _run(world, case)
+    got = _run(world, case, chunk=chunk)
     Q, K, V = _inputs(B, H, L, d, 17 + world)
     ref, keep, _ = oracle.forward(Q, K, V, tau, blk, blk, n_force)
     assert not keep.all()  # the thresholds skip blocks, so the correction takes part
@@ -102,8 +108,10 @@ def test_context_parallel_equals_the_single_process_oracle(world, H, lens, n_for
     assert np.array_equal(full, ref)
 
 
-def test_shape_mismatch_is_reported_on_every_rank():
-    # rank 1 passes one head fewer than rank 0: both see the gathered shapes and raise together
+@pytest.mark.parametrize("mismatch", ["heads", "k_shape"])
+def test_shape_mismatch_is_reported_on_every_rank(mismatch):
+    # rank 1 passes one head fewer, or a K shorter than its Q: every rank sees the gathered shapes
+    # and raises before any exchange, so none is left waiting in a collective
     case = (1, 4, 700, 16, 64, 0, [300, 400], [0.5] * 4, 3)
-    got = _run(2, case, mismatch=True)
+    got = _run(2, case, mismatch=mismatch)
     assert all(isinstance(got[r], str) and got[r].startswith("ValueError") for r in range(2)), got
