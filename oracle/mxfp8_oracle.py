@@ -3,9 +3,10 @@
 TEST INFRASTRUCTURE ONLY. Only the test-suite, the package's smoke check and the benchmark's
 CPU-baseline leg may import this module. The CUDA library never calls it and shares no code with it.
 
-The variant the pages point to: the Sol-Engine guide page (section on quantization) lists
-SageAttention, 8-bit to 4-bit attention with outlier smoothing, and a Sol-Engine news item
-reports "fused MXFP8 compute" for a B300 deployment. Neither prints a formula, so this oracle takes
+The variant the pages point to: the review page of the Sol Video Inference Engine paper lists
+SageAttention under quantization ("five acceleration techniques"): 8-bit to 4-bit attention with
+outlier smoothing. A Sol-Engine README news item reports "fused MXFP8 compute" for a B300
+deployment. Neither prints a formula, so this oracle takes
 the plainest reading that a Blackwell block-scaled tensor-core kernel computes:
 
 * Format: OCP Microscaling (MX) with FP8 E4M3 elements. Blocks of 32 consecutive values along
