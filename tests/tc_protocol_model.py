@@ -1,0 +1,229 @@
+"""Discrete-event model of the mbarrier protocol of the fused tensor-core kernel (one CTA).
+
+The model follows ``block_sparse_attention_41_b200/csrc/fwd_tc.cu`` role by role. It has the TMA
+producer, the QK^T issuer, the two PV issuers and the two softmax groups, each split into its
+waits, arrivals and commits, over a sequence of work units of T tiles each. Copies and MMAs
+complete after random delays. A run fails on:
+- a deadlock: no role can move and nothing is in flight;
+- a stale wait: a role waits for phase k of a barrier that has already completed phase k+1,
+  so its parity test would block or pass wrongly;
+- a hazard: a QK^T writing an S buffer whose P has not been consumed, a PV reading the wrong
+  tile's P or V, a copy overwriting a K/V stage still being read, an O rescale or read with a PV
+  in flight.
+
+Barrier semantics: a barrier of count c completes a phase after c arrivals; a wait for phase k
+(parity k & 1) passes once k + 1 phases have completed.
+"""
+from __future__ import annotations
+
+import random
+
+
+class Bar:
+    def __init__(self, name: str, count: int):
+        self.name, self.count, self.pending, self.n = name, count, 0, 0
+
+    def arrive(self):
+        self.pending += 1
+        if self.pending == self.count:
+            self.pending = 0
+            self.n += 1
+
+
+class Protocol:
+    """One CTA running `plan` (tiles per unit) with the kernel's K and V ring depths."""
+
+    def __init__(self, plan, seed, nk=3, nv=2, mutation=None):
+        self.plan, self.nk, self.nv, self.mut = plan, nk, nv, mutation
+        self.rng = random.Random(seed)
+        self.now, self.seq, self.events = 0, 0, []
+        pv_count = 1 if mutation == "pvdone_count_1" else 2
+        self.B = {"q": Bar("q", 1), "ofinal": Bar("ofinal", 2), "list": Bar("list", 1)}
+        for s in range(nk):
+            self.B[f"kfull{s}"], self.B[f"kempty{s}"] = Bar(f"kfull{s}", 1), Bar(f"kempty{s}", 1)
+        for s in range(nv):
+            self.B[f"vfull{s}"], self.B[f"vempty{s}"] = Bar(f"vfull{s}", 1), Bar(f"vempty{s}", 2)
+        for b in range(2):
+            self.B[f"sfull{b}"] = Bar(f"sfull{b}", 1)
+            self.B[f"pvdone{b}"] = Bar(f"pvdone{b}", pv_count)
+            for grp in range(2):
+                self.B[f"pfull{b}{grp}"] = Bar(f"pfull{b}{grp}", 1)
+        self.S = [None, None]          # (kind, tile, consumed): ("S", g) after QK(g), ("P", g) after softmax
+        self.S_busy = [set(), set()]   # MMAs in flight on each S buffer
+        self.halves = {}               # (buffer, tile) -> groups whose PV has completed
+        self.K = [None] * nk
+        self.V = [None] * nv
+        self.O_busy = [0, 0]           # PVs in flight per accumulator
+
+    # ---- event machinery
+    def later(self, fn):
+        self.seq += 1
+        self.events.append((self.now + self.rng.choice([1, 2, 5, 20, 60]), self.seq, fn))
+
+    def run(self):
+        roles = {"producer": self.producer(), "qk": self.qk_issuer(), "pv0": self.pv_issuer(0),
+                 "pv1": self.pv_issuer(1), "sm0": self.softmax(0), "sm1": self.softmax(1)}
+        waiting = dict.fromkeys(roles)
+        done, at_sync = set(), set()
+        while True:
+            moved = True
+            while moved:
+                moved = False
+                for name, gen in roles.items():
+                    if name in done or name in at_sync:
+                        continue
+                    if waiting[name] is not None:
+                        bar, k = waiting[name]
+                        if bar.n > k + 1:
+                            raise AssertionError(f"stale wait: {name} waits phase {k} of {bar.name}, at {bar.n}")
+                        if bar.n != k + 1:
+                            continue
+                        waiting[name] = None
+                    try:
+                        cmd = next(gen)
+                    except StopIteration:
+                        done.add(name)
+                        moved = True
+                        continue
+                    moved = True
+                    if cmd[0] == "wait":
+                        waiting[name] = (self.B[cmd[1]], cmd[2])
+                    else:  # "sync": the CTA-wide barrier at the end of a unit
+                        at_sync.add(name)
+                if at_sync and len(at_sync) == len(roles):
+                    at_sync.clear()
+                    moved = True
+            if len(done) == len(roles):
+                return
+            if not self.events:
+                raise AssertionError("deadlock: " + ", ".join(
+                    f"{n} waits {w[0].name}[{w[1]}]" for n, w in waiting.items() if w))
+            self.events.sort()
+            self.now, _, fn = self.events.pop(0)
+            fn()
+
+    # ---- roles
+    def producer(self):
+        base = 0
+        for u, T in enumerate(self.plan):
+            self.later(self.B["q"].arrive)
+            yield ("wait", "list", u)
+            for t in range(T + 1):
+                if t < T:
+                    g = base + t
+                    s = g % self.nk
+                    if g >= self.nk:
+                        yield ("wait", f"kempty{s}", g // self.nk - 1)
+
+                    def load_k(s=s, g=g):
+                        self.K[s] = g
+                        self.B[f"kfull{s}"].arrive()
+                    self.later(load_k)
+                if t >= 1:
+                    g = base + t - 1
+                    s = g % self.nv
+                    if g >= self.nv:
+                        yield ("wait", f"vempty{s}", g // self.nv - (2 if self.mut == "vempty_one_back" else 1))
+
+                    def load_v(s=s, g=g):
+                        self.V[s] = g
+                        self.B[f"vfull{s}"].arrive()
+                    self.later(load_v)
+            yield ("sync",)
+            base += T
+
+    def qk_issuer(self):
+        base = 0
+        for u, T in enumerate(self.plan):
+            yield ("wait", "list", u)
+            yield ("wait", "q", u)
+            for t in range(T):
+                g = base + t
+                b, s = g & 1, g % self.nk
+                if t >= 2 and self.mut != "qk_skips_pvdone":
+                    yield ("wait", f"pvdone{b}", (g - 2) >> 1)
+                yield ("wait", f"kfull{s}", g // self.nk)
+                if self.S_busy[b]:
+                    raise AssertionError(f"hazard: QK({g}) writes S{b} while {sorted(self.S_busy[b])} run")
+                if self.S[b] is not None and self.S[b][0] == "P" and not self.S[b][2]:
+                    raise AssertionError(f"hazard: QK({g}) overwrites P({self.S[b][1]}) before its PVs completed")
+                if self.K[s] != g:
+                    raise AssertionError(f"hazard: QK({g}) reads K stage {s} holding tile {self.K[s]}")
+                self.S_busy[b].add(("QK", g))
+
+                def qk_done(b=b, s=s, g=g):
+                    self.S_busy[b].discard(("QK", g))
+                    self.S[b] = ("S", g, False)
+                    self.B[f"sfull{b}"].arrive()
+                    self.B[f"kempty{s}"].arrive()
+                self.later(qk_done)
+            yield ("sync",)
+            base += T
+
+    def pv_issuer(self, grp):
+        base = 0
+        for u, T in enumerate(self.plan):
+            yield ("wait", "list", u)
+            for t in range(T):
+                g = base + t
+                b, s = g & 1, g % self.nv
+                yield ("wait", f"pfull{b}{grp}", g >> 1)
+                yield ("wait", f"vfull{s}", g // self.nv)
+                if self.S[b] is None or self.S[b][:2] != ("P", g):
+                    raise AssertionError(f"hazard: PV{grp}({g}) finds {self.S[b]} in S{b}")
+                if self.V[s] != g:
+                    raise AssertionError(f"hazard: PV{grp}({g}) reads V stage {s} holding tile {self.V[s]}")
+                self.S_busy[b].add(("PV", g, grp))
+                self.O_busy[grp] += 1
+
+                def pv_done(b=b, s=s, g=g):
+                    self.S_busy[b].discard(("PV", g, grp))
+                    self.O_busy[grp] -= 1
+                    if self.V[s] != g:
+                        raise AssertionError(f"hazard: V stage {s} overwritten during PV({g})")
+                    self.halves.setdefault((b, g), set()).add(grp)
+                    if self.halves[(b, g)] == {0, 1}:
+                        self.S[b] = ("P", g, True)
+                    self.B[f"vempty{s}"].arrive()
+                    self.B[f"pvdone{b}"].arrive()
+                self.later(pv_done)
+
+            def final_commit():
+                if self.O_busy[grp]:  # a commit arrives once this thread's MMAs have completed
+                    self.later(final_commit)
+                else:
+                    self.B["ofinal"].arrive()
+            self.later(final_commit)
+            yield ("sync",)
+            base += T
+
+    def softmax(self, grp):
+        base = 0
+        for u, T in enumerate(self.plan):
+            if grp == 0:
+                self.B["list"].arrive()  # thread 0 of the softmax warps publishes the tile lists
+            else:
+                yield ("wait", "list", u)
+            for t in range(T):
+                g = base + t
+                b = g & 1
+                yield ("wait", f"sfull{b}", g >> 1)
+                if self.S[b] is None or self.S[b][:2] not in (("S", g), ("P", g)):
+                    raise AssertionError(f"hazard: softmax{grp}({g}) finds {self.S[b]} in S{b}")
+                if t > 0 and self.rng.random() < 0.3:
+                    # a lazy rescale of O_grp: wait for the previous tile's PVs, then O_grp must be at rest
+                    yield ("wait", f"pvdone{(g - 1) & 1}", (g - 1) >> 1)
+                    if self.O_busy[grp]:
+                        raise AssertionError(f"hazard: rescale of O{grp} at tile {g} with a PV in flight")
+                self.S[b] = ("P", g, False)
+                self.B[f"pfull{b}{grp}"].arrive()
+            if T > 0:
+                yield ("wait", "ofinal", u)
+                if any(self.O_busy):
+                    raise AssertionError("hazard: the epilogue reads O with a PV in flight")
+            yield ("sync",)
+            base += T
+
+
+def random_plan(rng):
+    return [rng.choice([1, 1, 2, 3, 4, 5, 7, 8, 13]) for _ in range(rng.randint(1, 6))]

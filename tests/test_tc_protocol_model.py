@@ -1,0 +1,32 @@
+"""The fused kernel's mbarrier protocol, run as a discrete-event model (tests/tc_protocol_model.py).
+
+Random unit sizes (including one-tile units) and random completion delays, for the ring depths
+of both head dimensions: no deadlock, no stale parity wait, no data hazard. Three planted protocol
+mistakes must each be caught: a QK^T that does not wait for the PVs two tiles back, a PV-done
+barrier completed by one group instead of both, and a producer that waits for the V stage's
+use before the previous one.
+"""
+import random
+
+import pytest
+
+from tc_protocol_model import Protocol, random_plan
+
+
+@pytest.mark.parametrize("nk,nv", [(3, 2), (4, 4)])  # d = 128 and d = 64 ring depths
+def test_protocol_has_no_deadlock_stale_wait_or_hazard(nk, nv):
+    rng = random.Random(nk * 10 + nv)
+    for k in range(150):
+        Protocol(random_plan(rng), seed=k, nk=nk, nv=nv).run()
+
+
+@pytest.mark.parametrize("mutation", ["qk_skips_pvdone", "pvdone_count_1", "vempty_one_back"])
+def test_planted_protocol_mistakes_are_caught(mutation):
+    rng = random.Random(5)
+    caught = 0
+    for k in range(150):
+        try:
+            Protocol(random_plan(rng), seed=k, mutation=mutation).run()
+        except AssertionError:
+            caught += 1
+    assert caught > 0
