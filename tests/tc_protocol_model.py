@@ -33,8 +33,9 @@ class Bar:
 class Protocol:
     """One CTA running `plan` (tiles per unit) with the kernel's K and V ring depths."""
 
-    def __init__(self, plan, seed, nk=3, nv=2, mutation=None):
+    def __init__(self, plan, seed, nk=3, nv=2, mutation=None, route_in_kernel=False):
         self.plan, self.nk, self.nv, self.mut = plan, nk, nv, mutation
+        self.route_in_kernel = route_in_kernel  # no keep bits given: the softmax warps route from the Q tile
         self.rng = random.Random(seed)
         self.now, self.seq, self.events = 0, 0, []
         pv_count = 1 if mutation == "pvdone_count_1" else 2
@@ -200,6 +201,8 @@ class Protocol:
     def softmax(self, grp):
         base = 0
         for u, T in enumerate(self.plan):
+            if self.route_in_kernel:
+                yield ("wait", "q", u)  # q_bar comes from the Q tile in shared memory
             if grp == 0:
                 self.B["list"].arrive()  # thread 0 of the softmax warps publishes the tile lists
             else:

@@ -14,10 +14,11 @@ from tc_protocol_model import Protocol, random_plan
 
 
 @pytest.mark.parametrize("nk,nv", [(3, 2), (4, 4)])  # d = 128 and d = 64 ring depths
-def test_protocol_has_no_deadlock_stale_wait_or_hazard(nk, nv):
+@pytest.mark.parametrize("route_in_kernel", [False, True])  # keep bits from the routing pass, or routed in place
+def test_protocol_has_no_deadlock_stale_wait_or_hazard(nk, nv, route_in_kernel):
     rng = random.Random(nk * 10 + nv)
     for k in range(150):
-        Protocol(random_plan(rng), seed=k, nk=nk, nv=nv).run()
+        Protocol(random_plan(rng), seed=k, nk=nk, nv=nv, route_in_kernel=route_in_kernel).run()
 
 
 @pytest.mark.parametrize("mutation", ["qk_skips_pvdone", "pvdone_count_1", "vempty_one_back"])
