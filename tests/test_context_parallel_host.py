@@ -115,3 +115,16 @@ def test_shape_mismatch_is_reported_on_every_rank(mismatch):
     case = (1, 4, 700, 16, 64, 0, [300, 400], [0.5] * 4, 3)
     got = _run(2, case, mismatch=mismatch)
     assert all(isinstance(got[r], str) and got[r].startswith("ValueError") for r in range(2)), got
+
+
+def test_default_attention_is_the_cuda_path_with_no_cpu_fallback():
+    # one gloo rank, CPU tensors: the exchange works, and the default attention call refuses them
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    dist.init_process_group("gloo", rank=0, world_size=1)
+    try:
+        x = torch.zeros(1, 2, 64, 16)
+        with pytest.raises(TypeError, match="CUDA tensor"):
+            cp.sol_attn_context_parallel(x, x, x, [0.5, 0.5], block=64)
+    finally:
+        dist.destroy_process_group()
