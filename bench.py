@@ -428,13 +428,16 @@ def run_ours(args, w):
     dens = torch.empty((B, H), dtype=torch.float32, device=dev)
 
     def step(tau_v, ev=None):
-        sa.sol_attn_pool(K, V, blk, kbar, vbar, klp, vlp, stream=stream)
+        # ev: events before the pool kernel, between the pool kernel and the forward, after the forward
         if ev is not None:
             ev[0].record(stream)
+        sa.sol_attn_pool(K, V, blk, kbar, vbar, klp, vlp, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
         sa.sol_attn_fwd(Q, K, V, kbar, vbar, klp, vlp, tau_v, blk, blk, w.n_force, O=O, density=dens,
                         workspace=ws, stream=stream)
         if ev is not None:
-            ev[1].record(stream)
+            ev[2].record(stream)
 
     # kept blocks at the timed density (from the kernel's own density output)
     step(tau)
@@ -449,7 +452,7 @@ def run_ours(args, w):
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
-    fwd_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    fwd_ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_gpu_index(torch, local)) as clk:
         t0.record(stream)
@@ -466,7 +469,8 @@ def run_ours(args, w):
     gpu_rows = {(b, h, i): O[b, h, i * blk: (i + 1) * blk].double().cpu().numpy() for b, h, i in cpu_units}
     ms_total = max_over_ranks(t0.elapsed_time(t1))
     ms_step = ms_total / args.steps
-    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_ev)
+    fwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in fwd_ev)
+    pool_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in fwd_ev)
     value = world * flops / (ms_step * 1e-3) / 1e12
     pk = peaks()
     achieved = flops / (fwd_ms * 1e-3) / 1e12
@@ -480,14 +484,14 @@ def run_ours(args, w):
             torch.cuda.synchronize()
             kb = int(round(float(dens.double().sum()) * nb * nb))
             n_it = 3
-            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_it)]
+            evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(n_it)]
             a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a0.record(stream)
             for i in range(n_it):
                 step(tv, evs[i])
             a1.record(stream)
             torch.cuda.synchronize()
-            f_ms = statistics.mean(x.elapsed_time(y) for x, y in evs)
+            f_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
             sweep.append({"density_target": kk, "density": kb / float(B * H * nb * nb),
                           "ms_per_step": a0.elapsed_time(a1) / n_it, "fwd_ms": f_ms,
                           "fwd_tflops": kept_tile_flops(kb, w) / (f_ms * 1e-3) / 1e12})
@@ -546,6 +550,8 @@ def run_ours(args, w):
     per_run.pop("_mask_rows", None)
 
     traffic = captured_traffic(w, key)
+    # pooling reads K and V once and writes the fp32 means and their bf16 mirrors
+    pool_bytes = 2 * K.numel() * K.element_size() + 2 * B * H * nb * d * (4 + 2)
 
     if rank == 0:
         clocks = clk.summary()
@@ -566,6 +572,9 @@ def run_ours(args, w):
                                   "faster; the ncu launch list gives the split)",
                          "fwd_ms": fwd_ms,
                          "peak_source": f"{pk['source']} bf16 dense (burst)"},
+            "pool": {"kernel": "sol_pool_kernel", "ms": pool_ms, "algorithmic_bytes": pool_bytes,
+                     "GB/s": pool_bytes / (pool_ms * 1e-3) / 1e9, "bound": "hbm", "peak_GB/s": pk["hbm_gbs"],
+                     "frac": pool_bytes / (pool_ms * 1e-3) / 1e9 / pk["hbm_gbs"]},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 3 * args.steps,  # pool, routing pass, fused forward
