@@ -5,13 +5,16 @@ this package. The CUDA library never calls it.
 """
 from .sol_attn_oracle import (  # noqa: F401
     BAND,
+    adopt_in_band,
     band_mask,
     block_counts,
     forward,
     forward_head,
     pool_blocks,
+    proxy_error_bound,
     proxy_scores,
     route,
+    routing_violations,
     unit_forward,
     unit_terms,
 )

@@ -143,10 +143,9 @@ def forward_head(Q, K, V, tau, block_q, block_k, n_force=0, units=None, keep_ove
         qbar = rows.sum(axis=0) / nq[i]
         sbar = proxy_scores(qbar, kbar, d)
         kp, M = route(sbar, tau, n_force)
-        if keep_override is not None and not math.isinf(tau):
-            band = np.abs(sbar - (M - tau)) < BAND
-            band[: min(n_force, nkb)] = False
-            kp = np.where(band, keep_override[i], kp)
+        if keep_override is not None:
+            band = band_mask(sbar[None, :], np.array([M]), tau, n_force)[0]
+            kp = adopt_in_band(kp, band, keep_override[i])
         keep[i] = kp
         sbar_all[i] = sbar
         M_all[i] = M
@@ -171,9 +170,96 @@ def forward(Q, K, V, tau, block_q, block_k, n_force=0):
 
 
 def band_mask(sbar, M, tau, n_force=0):
-    """Entries whose routing decision lies within BAND of the threshold (never forced ones)."""
+    """Entries whose routing decision lies within BAND of the threshold (never forced ones).
+
+    sbar is [units, N_kb] and M [units]. At tau = +inf the threshold is -inf and no entry is
+    near it.
+    """
     if math.isinf(tau):
         return np.zeros_like(sbar, dtype=bool)
-    band = np.abs(sbar - (M[:, None] - tau)) < BAND
+    band = np.abs(sbar - (np.asarray(M, dtype=np.float64)[:, None] - tau)) < BAND
     band[:, : n_force] = False
     return band
+
+
+def adopt_in_band(keep, band, override):
+    """The oracle's routing decisions with `override` taken where `band` is set, and only there."""
+    return np.where(band, np.asarray(override, dtype=bool), keep)
+
+
+# ---------------------------------------------------------------------------------------------
+# Which kept sets a float32 evaluation of definition 2 may produce
+# ---------------------------------------------------------------------------------------------
+
+U32 = 2.0 ** -24  # unit roundoff of float32 (round to nearest)
+
+
+def _gamma(n: int) -> float:
+    """gamma_n = n u / (1 - n u): the relative bound of an n-operation float32 sum (Higham, 3.1)."""
+    return n * U32 / (1.0 - n * U32)
+
+
+def proxy_error_bound(Q, K, block_q, block_k, units=None):
+    """Upper bound on |s_fp32 - s_bar| for a float32 evaluation of definition 2 in ANY order.
+
+    The float32 pipeline: q_bar and k_bar are float32 sums of the m (n) valid rows of a block,
+    then one division or multiplication by the count; s is a float32 dot product of d terms,
+    then one multiplication by a rounded 1/sqrt(d). With A_c = mean_r |q_rc| over the query
+    block and B_jc = mean_t |k_tc| over key block j, the standard summation bound gives
+        |s_fp32 - s_bar| <= [(1 + g_{m+1})(1 + g_{n+1})(1 + g_d)(1 + 3u) - 1] * sum_c A_c B_jc / sqrt(d),
+    g_k = gamma_k: each float32 level is exact up to a relative factor of its absolute-value
+    sum, and those sums are bounded by A and B. Inputs are assumed exactly representable in
+    float32 (bf16 or float32 tensors). Returns [N_qb, N_kb] (rows outside `units` are NaN).
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    L, d = Q.shape
+    nqb, nq = block_counts(L, block_q)
+    nkb, nk = block_counts(K.shape[0], block_k)
+    B = pool_blocks(np.abs(K), block_k)  # [N_kb, d]
+    units = range(nqb) if units is None else units
+    eps = np.full((nqb, nkb), np.nan)
+    g_k = np.array([_gamma(int(n) + 1) for n in nk])
+    for i in units:
+        A = np.abs(Q[i * block_q: i * block_q + nq[i]]).sum(axis=0) / nq[i]
+        rel = (1 + _gamma(int(nq[i]) + 1)) * (1 + g_k) * (1 + _gamma(d)) * (1 + 3 * U32) - 1
+        eps[i] = rel * (B @ A) / math.sqrt(d)
+    return eps
+
+
+def routing_violations(sbar, M, tau, mask, eps, n_force=0):
+    """Check that `mask` is a kept set a float32 evaluation of definition 2 could produce.
+
+    sbar, eps, mask: [units, N_kb] (float64 scores, their float32 error bounds, the kept set under
+    test); M: [units]. For a float32 evaluation s~ with |s~ - s_bar| <= eps, the threshold
+    routing keeps j iff s~_j >= fl(M~ - tau) (or j is forced). Whatever the rounding, that gives:
+      forced      : every j < n_force is kept;
+      outside_band: outside the band |s_bar - (M - tau)| < BAND the decision equals the oracle's;
+      max_kept    : the float32 argmax is kept (fl(M~ - tau) <= M~ for tau >= 0), so some kept j
+                    has s_bar_j + eps_j >= M - eps_{argmax};
+      threshold   : a kept set of a threshold is upward closed in s~, so every non-forced kept j
+                    and skipped k satisfy s_bar_j + eps_j >= s_bar_k - eps_k.
+    Returns the number of rows (entries for the first two) that break each condition.
+    """
+    sbar = np.asarray(sbar, dtype=np.float64)
+    eps = np.asarray(eps, dtype=np.float64)
+    mask = np.asarray(mask, dtype=bool)
+    M = np.asarray(M, dtype=np.float64)
+    nf = min(n_force, sbar.shape[1])
+    keep_ref = sbar >= (M[:, None] - tau)
+    keep_ref[:, :nf] = True
+    band = band_mask(sbar, M, tau, n_force)
+    out = {"forced": int((~mask[:, :nf]).sum()),
+           "outside_band": int((mask[~band] != keep_ref[~band]).sum()),
+           "max_kept": 0, "threshold": 0}
+    for r in range(sbar.shape[0]):
+        s, e, m = sbar[r], eps[r], mask[r]
+        jstar = int(np.argmax(s))
+        if not m.any() or np.max(np.where(m, s + e, -np.inf)) < M[r] - e[jstar]:
+            out["max_kept"] += 1
+        free = np.arange(s.size) >= nf
+        kept, skipped = m & free, ~m
+        if kept.any() and skipped.any():
+            if np.min((s + e)[kept]) < np.max((s - e)[skipped]):
+                out["threshold"] += 1
+    return out

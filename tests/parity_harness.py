@@ -75,17 +75,27 @@ def _oracle_job(args):
     O, keep, sbar, M = oracle.forward_head(q, k, v, tau, w.block, w.block, n_force, units=qbs,
                                            keep_override=override)
     band = oracle.band_mask(sbar, M, tau, n_force)
+    eps = oracle.proxy_error_bound(q, k, w.block, w.block, units=qbs)
+    viol = oracle.routing_violations(sbar[qbs], M[qbs], tau, override[qbs], eps[qbs], n_force)
     out = []
     for i in qbs:
         rows = slice(i * w.block, min((i + 1) * w.block, w.L))
         out.append((i, O[rows], keep[i], band[i]))
-    return b, h, out
+    return b, h, out, viol
+
+
+def merge_violations(total, v):
+    for key, n in v.items():
+        total[key] = total.get(key, 0) + n
+    return total
 
 
 def compare_units(w, tau, units, O_gpu, mask_gpu, n_force=0):
     """Oracle vs CUDA path on the listed (b, h, i) units. The mask is compared bit for bit outside
-    the near-threshold band; O is compared after the oracle adopts the GPU's decision for band
-    entries. Returns a dict of error statistics."""
+    the near-threshold band, and every mask row must be a kept set that a float32 evaluation of the
+    routing could produce (oracle.routing_violations: forced blocks kept, the argmax kept, the kept
+    set closed upward in the score up to the float32 error bound). O is compared after the oracle
+    adopts the GPU's decision for band entries. Returns a dict of error statistics."""
     blk = w.block
     by_head = {}
     for b, h, i in units:
@@ -94,8 +104,10 @@ def compare_units(w, tau, units, O_gpu, mask_gpu, n_force=0):
     jobs = [(w.name, b, h, float(tau[h]), n_force, sorted(qbs), [mask_host[b, h, i] for i in sorted(qbs)])
             for (b, h), qbs in sorted(by_head.items())]
     max_err, sum_err, count, band_total, mism = 0.0, 0.0, 0, 0, 0
+    viol = {}
     with _pool(_workers(len(jobs))) as ex:
-        for b, h, res in ex.map(_oracle_job, jobs):
+        for b, h, res, v in ex.map(_oracle_job, jobs):
+            merge_violations(viol, v)
             for i, O_ref, keep_ref, band in res:
                 g = mask_host[b, h, i]
                 mism += int((g[~band] != keep_ref[~band]).sum())
@@ -106,7 +118,7 @@ def compare_units(w, tau, units, O_gpu, mask_gpu, n_force=0):
                 sum_err += float(err.sum())
                 count += err.size
     return {"max_abs": max_err, "mean_abs": sum_err / max(count, 1), "mask_mismatch_outside_band": mism,
-            "band_entries": band_total, "units": len(units)}
+            "band_entries": band_total, "units": len(units), "routing_violations": viol}
 
 
 def run_path(Q, K, V, tau, block, n_force=0):

@@ -20,8 +20,8 @@ from block_sparse_attention_41_b200 import sol_attn as sa
 from block_sparse_attention_41_b200 import workloads as wl
 from block_sparse_attention_41_b200.workloads import round_to_bf16
 
-from parity_harness import (TOL_BF16_MAX, TOL_BF16_MEAN, TOL_F32_MAX, compare_units, device_inputs, run_path,
-                            taus)
+from parity_harness import (TOL_BF16_MAX, TOL_BF16_MEAN, TOL_F32_MAX, compare_units, device_inputs,
+                            merge_violations, run_path, taus)
 
 pytestmark = pytest.mark.gpu
 
@@ -37,11 +37,20 @@ def _lib():
 
 def report(name, st):
     print(f"\n[{name}] max_abs={st['max_abs']:.3e} mean_abs={st['mean_abs']:.3e} "
-          f"band={st['band_entries']} mismatches={st['mask_mismatch_outside_band']} units={st['units']}")
+          f"band={st['band_entries']} mismatches={st['mask_mismatch_outside_band']} units={st['units']} "
+          f"routing_violations={st['routing_violations']}")
+
+
+def check_routing(st):
+    """The mask equals the oracle's outside the band and, inside it, is a kept set that a float32
+    evaluation of the routing could produce (every count of oracle.routing_violations is 0)."""
+    assert st["mask_mismatch_outside_band"] == 0
+    assert set(st["routing_violations"]) == {"forced", "outside_band", "max_kept", "threshold"}
+    assert all(n == 0 for n in st["routing_violations"].values()), st["routing_violations"]
 
 
 def check_bf16(st):
-    assert st["mask_mismatch_outside_band"] == 0
+    check_routing(st)
     assert st["max_abs"] <= TOL_BF16_MAX
     assert st["mean_abs"] <= TOL_BF16_MEAN
 
@@ -91,7 +100,7 @@ def test_tiny_f32_workload_full(tau):
     units = [(b, h, i) for b in range(w.B) for h in range(w.H) for i in range(w.n_blocks)]
     st = compare_units(w, t, units, O, mask)
     report(f"tiny f32 tau={tau}", st)
-    assert st["mask_mismatch_outside_band"] == 0
+    check_routing(st)
     assert st["max_abs"] <= TOL_F32_MAX
     check_mask_density(mask, dens)
     if math.isinf(tau):
@@ -178,6 +187,7 @@ def local_inputs(B, H, L, d, seed, pos=2.0, dtype="bf16"):
 def full_compare(Qh, Kh, Vh, O, mask, tau, blk, n_force=0):
     B, H, L, d = Qh.shape
     max_err, sum_err, n, mism, band_n = 0.0, 0.0, 0, 0, 0
+    viol = {}
     mk = mask.cpu().numpy().astype(bool)
     Og = O.double().cpu().numpy()
     for b in range(B):
@@ -185,6 +195,8 @@ def full_compare(Qh, Kh, Vh, O, mask, tau, blk, n_force=0):
             O_ref, keep, sbar, M = oracle.forward_head(Qh[b, h], Kh[b, h], Vh[b, h], tau[h], blk, blk, n_force,
                                                        keep_override=mk[b, h])
             band = oracle.band_mask(sbar, M, tau[h], n_force)
+            eps = oracle.proxy_error_bound(Qh[b, h], Kh[b, h], blk, blk)
+            merge_violations(viol, oracle.routing_violations(sbar, M, tau[h], mk[b, h], eps, n_force))
             mism += int((mk[b, h][~band] != keep[~band]).sum())
             band_n += int(band.sum())
             e = np.abs(Og[b, h] - O_ref)
@@ -192,7 +204,7 @@ def full_compare(Qh, Kh, Vh, O, mask, tau, blk, n_force=0):
             sum_err += float(e.sum())
             n += e.size
     return {"max_abs": max_err, "mean_abs": sum_err / n, "mask_mismatch_outside_band": mism, "band_entries": band_n,
-            "units": B * H}
+            "units": B * H, "routing_violations": viol}
 
 
 @pytest.mark.parametrize("L", [1, 5, 100, 128, 129, 383, 1000, 2049])
@@ -277,11 +289,13 @@ def test_routing_pass_matches_in_kernel_routing(L, d, H):
         O_ref, keep, sbar, M = oracle.forward_head(Qh[0, 0], Kh[0, 0], Vh[0, 0], tau[0], 128, 128, 0, units=units,
                                                    keep_override=mk)
         band = oracle.band_mask(sbar[units], M[units], tau[0], 0)
+        eps = oracle.proxy_error_bound(Qh[0, 0], Kh[0, 0], 128, 128, units=units)
         rows = np.concatenate([np.arange(i * 128, min(L, i * 128 + 128)) for i in units])
         e = np.abs(O[0, 0].double().cpu().numpy()[rows] - O_ref[rows])
         st = {"max_abs": float(e.max()), "mean_abs": float(e.mean()),
               "mask_mismatch_outside_band": int((mk[units][~band] != keep[units][~band]).sum()),
-              "band_entries": int(band.sum()), "units": len(units)}
+              "band_entries": int(band.sum()), "units": len(units),
+              "routing_violations": oracle.routing_violations(sbar[units], M[units], tau[0], mk[units], eps[units])}
     report(f"routing pass L={L} d={d}", st)
     check_bf16(st)
 
@@ -294,7 +308,8 @@ def test_f32_path_shapes(blk, d):
     O, mask, dens = run_path(Q, K, V, tau, blk)
     st = full_compare(Qh, Kh, Vh, O, mask, tau, blk)
     report(f"f32 blk={blk} d={d}", st)
-    assert st["mask_mismatch_outside_band"] == 0 and st["max_abs"] <= TOL_F32_MAX
+    check_routing(st)
+    assert st["max_abs"] <= TOL_F32_MAX
     check_mask_density(mask, dens)
 
 
