@@ -284,6 +284,85 @@ def measure_qknorm_rope_pool(w, Q, K, V, stream, pk, cpu_ok, max_over_ranks, bar
     return out
 
 
+OTHER_CONFIGS = ("small_dit_L8192", "video1080p_L252960", "text_video_cfg_L33272")
+
+
+def measure_config(name, dev, stream, pk, parity_units=4):
+    """One of the other bf16 workloads at its target density: CUDA-event time of the sol_attn_fwd
+    call (routing pass + fused kernel), kept-tile TFLOP/s and its fraction of the bf16 peak, the
+    same call at tau = +inf (dense), the per-CTA busy spread of the persistent kernel, and a
+    sampled check of the timed output against the oracle."""
+    import torch
+    from block_sparse_attention_41_b200 import sol_attn as sa
+    w = wl.WORKLOADS[name]
+    Q, K, V = device_inputs(w, dev, torch)
+    key = density_keys(w)[0]
+    tau = tau_for(w, key)
+    B, H, L, d, blk, nb = w.B, w.H, w.L, w.d, w.block, w.n_blocks
+    ws = sa.new_workspace(B, H, L, blk, dev)
+    kbar, vbar, klp, vlp = sa.sol_attn_pool(K, V, blk, stream=stream)
+    O = torch.empty_like(Q)
+    dens = torch.empty((B, H), dtype=torch.float32, device=dev)
+    mask = torch.empty((B, H, nb, nb), dtype=torch.uint8, device=dev)
+
+    def fwd(tv, m=None):
+        sa.sol_attn_fwd(Q, K, V, kbar, vbar, klp, vlp, tv, blk, blk, w.n_force, O=O, kept_mask=m, density=dens,
+                        workspace=ws, stream=stream)
+
+    def timed(tv, n_it):
+        for _ in range(2):
+            fwd(tv)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_it)]
+        for a, b in ev:
+            a.record(stream)
+            fwd(tv)
+            b.record(stream)
+        torch.cuda.synchronize()
+        sa.sol_attn_check_device_error(ws)
+        return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+    fwd(tau, mask)
+    torch.cuda.synchronize()
+    kept = int(mask.to(torch.int64).sum())
+    flops = kept_tile_flops(kept, w)
+    ms = timed(tau, 5)
+    spans = cta_spans(lambda: fwd(tau), dev, torch, sa)
+    dense_ms = timed([math.inf] * H, 3)
+    fwd(tau)  # leave the timed density's output in O for the parity sample
+    torch.cuda.synchronize()
+    units = cpu_sample_units(w, parity_units, 91)
+    gpu_rows = {(b, h, i): O[b, h, i * blk: (i + 1) * blk].double().cpu().numpy() for b, h, i in units}
+    mask_rows = _rows_by_unit(mask, units)
+    collected = []
+    oracle_sample(w, tau, 1e9, max_units=parity_units, seed_offset=91, collect=collected)
+    achieved = flops / (ms * 1e-3) / 1e12
+    out = {"B": B, "H": H, "L": L, "d": d, "block": blk, "n_force": w.n_force, "density_target": key,
+           "density": kept / float(B * H * nb * nb), "kept_tiles": kept, "fwd_ms": ms, "fwd_tflops": achieved,
+           "frac": achieved / pk["bf16_tflops"], "dense_fwd_ms": dense_ms, "speedup_vs_dense": dense_ms / ms,
+           "cta_balance": spans, "parity_sample": sample_parity(collected, gpu_rows, mask_rows)}
+    del Q, K, V, O, ws, kbar, vbar, klp, vlp, mask
+    torch.cuda.empty_cache()
+    return out
+
+
+def cta_spans(launch, dev, torch, sa):
+    """Per-CTA start and finish times (globaltimer) of one fused-kernel launch, recorded by the
+    library's test hook: the tail is the last finish minus the mean finish, as a fraction of the
+    launch's span (first start to last finish)."""
+    buf = torch.zeros(2 * 4096, dtype=torch.int64, device=dev)
+    sa.sol_attn_debug_record_cta_times(buf, 4096)
+    launch()
+    torch.cuda.synchronize()
+    t = buf.view(-1, 2).cpu().numpy()
+    t = t[t[:, 1] > 0]
+    if t.size == 0:
+        return None
+    start, end = t[:, 0].astype(np.float64), t[:, 1].astype(np.float64)
+    span = end.max() - start.min()
+    return {"ctas": int(t.shape[0]), "span_ms": span * 1e-6, "tail_ms": (end.max() - end.mean()) * 1e-6,
+            "tail_frac": float((end.max() - end.mean()) / span), "busy_frac": float(((end - start) / span).mean())}
+
+
 def per_run_report(w, Q, K, V, kbar, vbar, klp, vlp, tau, key, O, dens, ws, stream):
     """One untimed call with the kept mask: per-head densities, kept-tile FLOPs over valid tokens
     only (the partial last query and key blocks count their valid rows and columns), the
@@ -552,6 +631,17 @@ def run_ours(args, w):
     traffic = captured_traffic(w, key)
     # pooling reads K and V once and writes the fp32 means and their bf16 mirrors
     pool_bytes = 2 * K.numel() * K.element_size() + 2 * B * H * nb * d * (4 + 2)
+    qkv_gb = 3 * Q.numel() * Q.element_size() / 1e9
+
+    configs = None
+    if not args.no_configs and world == 1:
+        configs = {w.name: {"fwd_ms": fwd_ms, "fwd_tflops": achieved, "frac": achieved / pk["bf16_tflops"],
+                            "cta_balance": cta_spans(lambda: step(tau), dev, torch, sa)}}
+        del Q, K, V, O, kbar, vbar, klp, vlp
+        torch.cuda.empty_cache()
+        for name in OTHER_CONFIGS:
+            if name != w.name:
+                configs[name] = measure_config(name, dev, stream, pk)
 
     if rank == 0:
         clocks = clk.summary()
@@ -562,8 +652,7 @@ def run_ours(args, w):
             "config": {"workload": w.name, "B": B, "H": H, "L": L, "d": d, "block": blk,
                        "density_target": key, "density": kept / float(B * H * nb * nb),
                        "kept_tiles": kept, "n_force": w.n_force,
-                       "l2": "inputs (Q,K,V %.2f GB) larger than the 126 MB L2; no flush" %
-                             (3 * Q.numel() * Q.element_size() / 1e9),
+                       "l2": "inputs (Q,K,V %.2f GB) larger than the 126 MB L2; no flush" % qkv_gb,
                        "parallelism": f"replica x{world}"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": achieved / pk["bf16_tflops"], "traffic": traffic,
@@ -582,6 +671,7 @@ def run_ours(args, w):
             "sweep": sweep,
             "next_rows": next_rows,
             "per_run": per_run,
+            "configs": configs,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -610,6 +700,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-next", action="store_true", help="skip the fused QK-norm + RoPE + pooling measurement")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other workloads (ms, roofline, dense ratio)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-budget", type=float, default=0.0,
                     help="reference arm: seconds of oracle work per step (default: fit a few minutes)")

@@ -119,6 +119,8 @@ struct TcParams {
   float log2_last_n;
   int drop_one_load;
   unsigned long long wait_limit_ns;
+  unsigned long long* cta_times;  // measurement hook: [2 * cta_capacity] start/finish ns, or null
+  int cta_capacity;
   float tau[kMaxHeads];
 };
 
@@ -218,6 +220,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + C::OFF_TMEM);
+  const bool stamp = p.cta_times != nullptr && static_cast<int>(blockIdx.x) < p.cta_capacity && tid == 0;
+  if (stamp) p.cta_times[2 * blockIdx.x] = globaltimer_ns();
 
   uint32_t tile_base = 0;  // tiles processed by this CTA before the current unit (all roles agree)
   uint32_t unit_iter = 0;  // units processed by this CTA before the current one
@@ -715,6 +719,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     ++unit_iter;
   }
 
+  if (stamp) p.cta_times[2 * blockIdx.x + 1] = globaltimer_ns();
+
   // ---- drain: no copy or MMA may still be in flight when TMEM and shared memory are released
   if ((warp == 1 || warp == kPv1Warp || warp == kQkWarp) && lane == 0 && mma_issued) {
     const uint32_t bd = bar_drain + (warp == 1 ? 0 : (warp == kPv1Warp ? 8 : 16));
@@ -770,6 +776,8 @@ cudaError_t launch_tc_t(const FwdArgs& a, const CUtensorMap* maps, cudaStream_t 
   p.log2_last_n = static_cast<float>(std::log2(static_cast<double>(p.last_n)));
   p.drop_one_load = a.drop_one_load;
   p.wait_limit_ns = a.wait_limit_ns;
+  p.cta_times = a.cta_times;
+  p.cta_capacity = a.cta_capacity;
   for (int h = 0; h < kMaxHeads; ++h) p.tau[h] = h < a.H ? a.tau[h] : 0.f;
   cudaError_t e = cudaFuncSetAttribute(sol_fwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_BYTES);

@@ -28,7 +28,11 @@ struct FwdArgs {
   int drop_one_load;       // failure-detection test hook (bf16 path)
   uint32_t* route_bits;    // bf16 path: [B*H, N_qb, ceil(N_kb/32)] keep bits from launch_route, or null
                            // (the fused kernel then routes each unit itself)
+  float* route_qbar;       // with route_bits: [B*H, N_qb, d] fp32 query-block means (workspace)
   uint64_t wait_limit_ns;  // bound on every on-device wait
+  int k_keep = 0;          // routing pass: 0 = threshold max - tau; k > 0 = the k highest scores
+  unsigned long long* cta_times = nullptr;  // measurement hook: [2 * cta_capacity] start/finish ns
+  int cta_capacity = 0;
 };
 
 cudaError_t launch_pool(const void* K, const void* V, bool bf16, int BH, int L, int d, int block,
@@ -55,8 +59,9 @@ struct RopePoolArgs {
 // bf16, d in {64, 128}: QK RMS norm + rotary embedding + K/V block pooling in one pass.
 cudaError_t launch_qknorm_rope_pool(const RopePoolArgs& a, cudaStream_t stream);
 
-// bf16, d in {64, 128}, block 128: routing pass for every unit; writes a.route_bits, the optional
-// mask and the per-head kept counts (ws + WS_COUNTS).
+// bf16, d in {64, 128}, block 128: routing pass for every unit (q_bar kernel, then the routing
+// kernel); writes a.route_qbar, a.route_bits, the optional mask and the per-head kept counts
+// (ws + WS_COUNTS).
 cudaError_t launch_route(const FwdArgs& a, cudaStream_t stream);
 
 // bf16, d in {64, 128}, block 128: TMA + tcgen05 persistent kernel.

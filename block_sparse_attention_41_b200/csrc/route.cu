@@ -1,11 +1,13 @@
 // Routing pass of the bf16 Sol-Attn forward (Sol-Attn project page, Abstract: the kept key blocks of
 // each query block are chosen on the fly by a query-dependent threshold on a cheap proxy score).
 //
-// For a run of R query blocks of one head, one CTA computes
-//   q_bar_i  = mean of the valid query rows of block i          (from Q in global memory)
+// Two kernels. The first, sol_qbar_kernel, streams Q once at full HBM bandwidth and writes
+//   q_bar_i  = mean of the valid query rows of block i          (fp32, into the workspace)
+// for every query block. The second, for a run of R query blocks of one head per CTA, computes
 //   s_bar_ij = q_bar_i . k_bar_j / sqrt(d) for every key block j  (fp32, shared memory only)
 //   keep_ij  = s_bar_ij >= max_j s_bar_ij - tau[h]  or  j < n_force
-// and writes only the keep bits (one u32 word per 32 key blocks), the optional uint8 mask, and the
+// or, in fixed-sparsity mode, keep_ij = j among the k highest s_bar_ij (equal scores: the lower
+// index first) or j < n_force, and writes only the keep bits (one u32 word per 32 key blocks), the optional uint8 mask, and the
 // per-head kept-block count. The proxy scores never leave shared memory.
 //
 // Doing this for R query blocks at once reads each head's pooled keys once per R units instead of
@@ -24,12 +26,13 @@ constexpr int kRouteWarps = kRouteThreads / 32;
 constexpr int kRows = 128;
 
 struct RouteParams {
-  const __nv_bfloat16* Q;  // [BH, L, D]
+  const float* qbar;       // [BH, nqb, D] fp32, from sol_qbar_kernel
   const float* kbar;       // [BH, nkb, D] fp32
   uint32_t* bits;          // [BH, nqb, nwords]
   uint8_t* kept_mask;      // [BH, nqb, nkb] or null
   uint32_t* counts;        // [BH] kept blocks per head (accumulated)
   int BH, H, L, nqb, nkb, nwords, n_force;
+  int k_keep;  // 0: threshold routing; k > 0: the k highest scores
   float inv_sqrt_d;
   float tau[kMaxHeads];
 };
@@ -61,12 +64,149 @@ __device__ __forceinline__ void butterfly_sum(float (&v)[N], int lane) {
   }
 }
 
+// A 32-bit key whose unsigned order is the order of the fp32 scores (-0 counted as +0).
+__device__ __forceinline__ uint32_t ordered_key(float f) {
+  const uint32_t u = __float_as_uint(f + 0.0f);  // -0 + 0 = +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// The lowest n set bits of m.
+__device__ __forceinline__ uint32_t lowest_bits(uint32_t m, int n) {
+  uint32_t r = 0;
+  for (int i = 0; i < n && m; ++i) {
+    const uint32_t b = m & (0u - m);
+    r |= b;
+    m ^= b;
+  }
+  return r;
+}
+
+// Key of the k-th highest of the nkb scores in sc (k >= 1), and how many scores equal to it are
+// among the k highest. One warp, a 256-bin histogram per 8 key bits, most significant first.
+__device__ __forceinline__ void radix_select_kth(const float* sc, int nkb, int k, uint32_t* hist, int lane,
+                                                 uint32_t* key_out, int* eq_out) {
+  uint32_t prefix = 0, pmask = 0;
+  int kk = k;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = lane; b < 256; b += 32) hist[b] = 0;
+    __syncwarp();
+    for (int j = lane; j < nkb; j += 32) {
+      const uint32_t key = ordered_key(sc[j]);
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
+    __syncwarp();
+    // lane l holds bins [8l, 8l + 8); count the candidates in higher bins, from the top
+    uint32_t c[8], lsum = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      c[q] = hist[8 * lane + q];
+      lsum += c[q];
+    }
+    uint32_t suf = lsum;  // candidates in lanes lane .. 31
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_down_sync(0xffffffffu, suf, o);
+      if (lane + o < 32) suf += y;
+    }
+    const uint32_t above = suf - lsum;
+    const bool mine = above < static_cast<uint32_t>(kk) && static_cast<uint32_t>(kk) <= suf;
+    const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+    int bin = 0;
+    uint32_t higher = 0;
+    if (mine) {
+      uint32_t acc = above;
+      int qsel = -1;
+#pragma unroll
+      for (int q = 7; q >= 0; --q) {  // the highest bin whose count reaches the k-th score
+        const bool hit = qsel < 0 && acc + c[q] >= static_cast<uint32_t>(kk);
+        if (hit) {
+          qsel = q;
+          higher = acc;
+        }
+        acc += c[q];
+      }
+      bin = 8 * lane + qsel;
+    }
+    bin = __shfl_sync(0xffffffffu, bin, src);
+    higher = __shfl_sync(0xffffffffu, higher, src);
+    prefix |= static_cast<uint32_t>(bin) << shift;
+    pmask |= 255u << shift;
+    kk -= static_cast<int>(higher);
+    __syncwarp();
+  }
+  *key_out = prefix;
+  *eq_out = kk;
+}
+
+// q_bar of QB query blocks of one head per CTA. Thread t sums one 16-byte chunk (8 columns) of a
+// block over the rows r = rg, rg + RG, ... in ascending order (rg = t / (D / 8), RG = 256 / (D / 8)),
+// then the RG partial sums of a column are added in the order rg = 0, 1, ... and divided by the
+// number of valid rows. The fused kernel's own routing (from its Q tile) takes exactly these
+// fp32 operations in this order, so both routing paths get the same q_bar bit for bit. All of a
+// thread's loads are issued before the first addition, so each CTA keeps QB * 16 KB (d = 128) of
+// Q in flight.
+template <int D, int QB>
+__global__ void __launch_bounds__(kRouteThreads) sol_qbar_kernel(const __nv_bfloat16* __restrict__ Q,
+                                                                 float* __restrict__ qbar, int L, int nqb) {
+  constexpr int CH = D / 8;
+  constexpr int RG = kRouteThreads / CH;
+  constexpr int RPT = kRows / RG;  // rows per thread and block
+  __shared__ float part[QB][RG][D];
+  const int tid = threadIdx.x;
+  const int bh = blockIdx.y;
+  const int qb0 = blockIdx.x * QB;
+  const int c8 = tid % CH, rg = tid / CH;
+  uint4 v[QB][RPT];
+  int m[QB];
+#pragma unroll
+  for (int b = 0; b < QB; ++b) {
+    m[b] = (qb0 + b < nqb) ? min(kRows, L - (qb0 + b) * kRows) : 0;
+    const __nv_bfloat16* base = Q + (static_cast<size_t>(bh) * L + static_cast<size_t>(qb0 + b) * kRows) * D + c8 * 8;
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+      const int r = rg + k * RG;
+      v[b][k] = r < m[b] ? __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(r) * D))
+                         : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+#pragma unroll
+  for (int b = 0; b < QB; ++b) {
+    float a[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = 0.f;
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+      if (rg + k * RG < m[b]) {
+        const uint32_t wv[4] = {v[b][k].x, v[b][k].y, v[b][k].z, v[b][k].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          a[2 * q] += __uint_as_float(wv[q] << 16);
+          a[2 * q + 1] += __uint_as_float(wv[q] & 0xffff0000u);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) part[b][rg][c8 * 8 + k] = a[k];
+  }
+  __syncthreads();
+  for (int idx = tid; idx < QB * D; idx += kRouteThreads) {
+    const int b = idx / D, c = idx % D;
+    if (m[b] > 0) {
+      float q = 0.f;
+#pragma unroll 8
+      for (int k = 0; k < RG; ++k) q += part[b][k][c];
+      qbar[(static_cast<size_t>(bh) * nqb + qb0 + b) * D + c] = q / static_cast<float>(m[b]);
+    }
+  }
+}
+
 template <int D, int R>
 __global__ void __launch_bounds__(kRouteThreads) sol_route_kernel(const __grid_constant__ RouteParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   float* s_qbar = reinterpret_cast<float*>(smem_raw);  // [R][D]
-  float* s_sc = s_qbar + R * D;                         // [R][nkb]; its start also holds the q_bar partials
+  float* s_sc = s_qbar + R * D;                         // [R][nkb] proxy scores
   __shared__ uint32_t s_cnt;
+  __shared__ uint32_t s_hist[kRouteWarps][256];  // fixed-sparsity mode: one histogram per warp
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.y;
@@ -75,59 +215,12 @@ __global__ void __launch_bounds__(kRouteThreads) sol_route_kernel(const __grid_c
   const int nkb = p.nkb;
   if (tid == 0) s_cnt = 0;
 
-  // (1) q_bar of each of the nr query blocks, four blocks at a time: thread t sums a 16-byte chunk
-  // (8 columns) of each over a strided set of rows (the same rows, in the same order, as the fused
-  // kernel's own routing); partial sums meet in shared memory
+  // (1) q_bar of the nr query blocks, from the workspace
   {
-    constexpr int CH = D / 8;
-    constexpr int RG = kRouteThreads / CH;
-    constexpr int NB = 4;
-    const int c8 = tid % CH, rg = tid / CH;
-    float* part = s_sc;  // [NB][RG][D]
-    for (int r0 = 0; r0 < nr; r0 += NB) {
-      float a[NB][8];
-      int m[NB];
-#pragma unroll
-      for (int rb = 0; rb < NB; ++rb) {
-        m[rb] = (r0 + rb < nr) ? min(kRows, p.L - (qb0 + r0 + rb) * kRows) : 0;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) a[rb][k] = 0.f;
-      }
-      const __nv_bfloat16* qrow = p.Q + (static_cast<size_t>(bh) * p.L + static_cast<size_t>(qb0 + r0) * kRows) * D + c8 * 8;
-#pragma unroll 2
-      for (int rr = rg; rr < kRows; rr += RG) {
-        uint4 v[NB];
-#pragma unroll
-        for (int rb = 0; rb < NB; ++rb)
-          if (rr < m[rb]) v[rb] = __ldg(reinterpret_cast<const uint4*>(qrow + static_cast<size_t>(rb * kRows + rr) * D));
-#pragma unroll
-        for (int rb = 0; rb < NB; ++rb) {
-          if (rr < m[rb]) {
-            const uint32_t wv[4] = {v[rb].x, v[rb].y, v[rb].z, v[rb].w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              a[rb][2 * k] += __uint_as_float(wv[k] << 16);
-              a[rb][2 * k + 1] += __uint_as_float(wv[k] & 0xffff0000u);
-            }
-          }
-        }
-      }
-#pragma unroll
-      for (int rb = 0; rb < NB; ++rb)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) part[(rb * RG + rg) * D + c8 * 8 + k] = a[rb][k];
-      __syncthreads();
-      for (int idx = tid; idx < NB * D; idx += kRouteThreads) {
-        const int rb = idx / D, c = idx % D;
-        if (r0 + rb < nr) {
-          float q = 0.f;
-          for (int k = 0; k < RG; ++k) q += part[(rb * RG + k) * D + c];
-          s_qbar[(r0 + rb) * D + c] = q / static_cast<float>(m[rb]);
-        }
-      }
-      __syncthreads();
-    }
+    const float* src = p.qbar + (static_cast<size_t>(bh) * p.nqb + qb0) * D;
+    for (int idx = tid; idx < nr * D; idx += kRouteThreads) s_qbar[idx] = src[idx];
   }
+  __syncthreads();
 
   // (2) proxy scores: warp w takes key blocks w, w + 8, ...; lane l holds components [l DPL, (l+1) DPL)
   {
@@ -177,8 +270,34 @@ __global__ void __launch_bounds__(kRouteThreads) sol_route_kernel(const __grid_c
   }
   __syncthreads();
 
-  // (3) per query block: max, threshold, keep bits, mask bytes, count (warp w takes blocks w, w + 8, ...)
-  {
+  // (3) per query block: max, threshold (or the k-th highest score), keep bits, mask bytes, count
+  // (warp w takes blocks w, w + 8, ...)
+  if (p.k_keep > 0) {
+    uint32_t kept = 0;
+    for (int r = warp; r < nr; r += kRouteWarps) {
+      const float* sc = s_sc + r * nkb;
+      uint32_t kth;
+      int take;  // scores equal to the k-th one still to keep, lowest index first
+      radix_select_kth(sc, nkb, p.k_keep, s_hist[warp], lane, &kth, &take);
+      const size_t unit = static_cast<size_t>(bh) * p.nqb + qb0 + r;
+      uint32_t* bw = p.bits + unit * p.nwords;
+      uint8_t* mrow = p.kept_mask != nullptr ? p.kept_mask + unit * nkb : nullptr;
+      for (int i = 0; i < p.nwords; ++i) {
+        const int j = 32 * i + lane;
+        const uint32_t key = j < nkb ? ordered_key(sc[j]) : 0u;
+        const uint32_t gt = __ballot_sync(0xffffffffu, j < nkb && key > kth);
+        const uint32_t eq = __ballot_sync(0xffffffffu, j < nkb && key == kth);
+        const uint32_t eq_kept = lowest_bits(eq, take);
+        take -= __popc(eq_kept);
+        const uint32_t forced = __ballot_sync(0xffffffffu, j < nkb && j < p.n_force);
+        const uint32_t m = gt | eq_kept | forced;
+        if (lane == 0) bw[i] = m;
+        if (mrow != nullptr && j < nkb) mrow[j] = static_cast<uint8_t>((m >> lane) & 1u);
+        kept += __popc(m);
+      }
+    }
+    if (lane == 0 && kept) atomicAdd(&s_cnt, kept);
+  } else {
     const float tau = p.tau[bh % p.H];
     uint32_t kept = 0;
     for (int r = warp; r < nr; r += kRouteWarps) {
@@ -209,7 +328,7 @@ __global__ void __launch_bounds__(kRouteThreads) sol_route_kernel(const __grid_c
 template <int D, int R>
 cudaError_t launch_route_t(const FwdArgs& a, cudaStream_t stream) {
   RouteParams p;
-  p.Q = static_cast<const __nv_bfloat16*>(a.Q);
+  p.qbar = a.route_qbar;
   p.kbar = a.kbar;
   p.bits = a.route_bits;
   p.kept_mask = a.kept_mask;
@@ -221,14 +340,16 @@ cudaError_t launch_route_t(const FwdArgs& a, cudaStream_t stream) {
   p.nkb = p.nqb;
   p.nwords = (p.nkb + 31) / 32;
   p.n_force = a.n_force;
+  p.k_keep = a.k_keep;
   p.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   for (int h = 0; h < kMaxHeads; ++h) p.tau[h] = h < a.H ? a.tau[h] : 0.f;
-  constexpr int RG = kRouteThreads / (D / 8);
-  const size_t part_floats = static_cast<size_t>(4) * RG * D;  // q_bar partial sums of four blocks
-  const size_t sc_floats = static_cast<size_t>(R) * p.nkb > part_floats ? static_cast<size_t>(R) * p.nkb : part_floats;
-  const size_t smem = (static_cast<size_t>(R) * D + sc_floats) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(sol_route_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  constexpr int QB = 2;
+  sol_qbar_kernel<D, QB><<<dim3((p.nqb + QB - 1) / QB, p.BH), kRouteThreads, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(a.Q), a.route_qbar, p.L, p.nqb);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = (static_cast<size_t>(R) * D + static_cast<size_t>(R) * p.nkb) * sizeof(float);
+  e = cudaFuncSetAttribute(sol_route_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const dim3 grid((p.nqb + R - 1) / R, p.BH);
   sol_route_kernel<D, R><<<grid, kRouteThreads, smem, stream>>>(p);

@@ -16,6 +16,8 @@ namespace {
 
 thread_local std::string g_last_error;
 int g_drop_one_load = 0;  // failure-detection test hook, consumed by the next bf16 launch
+unsigned long long* g_cta_times = nullptr;  // measurement hook, consumed by the next bf16 launch
+int g_cta_capacity = 0;
 
 sol_status fail(sol_status s, const char* fmt, ...) {
   char buf[512];
@@ -97,13 +99,40 @@ size_t ws_bits_bytes(int B, int H, int L, int block) {
   const size_t bytes = static_cast<size_t>(B) * H * nb * ((nb + 31) / 32) * 4;
   return (bytes + 255) / 256 * 256;
 }
+// After the keep bits: the routing pass's query-block means, fp32 [B*H][N_qb][d], sized for the
+// largest head dimension of the bf16 path (128) because the size function takes no d.
+constexpr size_t kQbarMaxD = 128;
+size_t ws_qbar_bytes(int B, int H, int L, int block) {
+  const size_t nb = (static_cast<size_t>(L) + block - 1) / block;
+  const size_t bytes = static_cast<size_t>(B) * H * nb * kQbarMaxD * 4;
+  return (bytes + 255) / 256 * 256;
+}
+size_t ws_route_bytes(int B, int H, int L, int block) { return ws_bits_bytes(B, H, L, block) + ws_qbar_bytes(B, H, L, block); }
 
 // ---- workspace in the library's own device memory, for sol_attn_fwd_noalloc -------------------
 constexpr int kNoAllocMaxHeads = 4096;  // B * H
-constexpr size_t kNoAllocWords = static_cast<size_t>(sol::WS_COUNTS) + kNoAllocMaxHeads;
+// the header of kNoAllocMaxHeads heads, rounded to 256 bytes as ws_header_bytes does (16,640 B)
+constexpr size_t kNoAllocBytes = ((static_cast<size_t>(sol::WS_COUNTS) + kNoAllocMaxHeads) * 4 + 255) / 256 * 256;
+constexpr size_t kNoAllocWords = kNoAllocBytes / 4;
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kMaxDevices] = {};
+void* g_noalloc_ctx[kMaxDevices] = {};  // the context the address was looked up in
+
+// cuCtxGetCurrent through the runtime's driver entry point (no link-time libcuda).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn() {
+  static std::once_flag once;
+  static CtxGetCurrentFn fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(f);
+  });
+  return fn;
+}
 
 }  // namespace
 
@@ -113,18 +142,26 @@ static __device__ __align__(256) uint32_t g_noalloc_ws[kNoAllocWords];
 
 namespace {
 
-// Device address of g_noalloc_ws on the current device, looked up once per device.
+// Device address of g_noalloc_ws on the current device. It is looked up once per device and
+// context: after a cudaDeviceReset the primary context, and with it the module that holds the
+// array, is created anew, so a changed current context triggers a fresh lookup.
 sol_status noalloc_workspace(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(SOL_EUNSUPPORTED, "device index %d beyond %d", dev, kMaxDevices);
+  CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+  if (get_ctx == nullptr) return fail(SOL_ECUDA, "cuCtxGetCurrent is not available from the driver");
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  CUcontext ctx = nullptr;  // null while the runtime has not yet made a context current here
+  if (get_ctx(&ctx) != CUDA_SUCCESS) ctx = nullptr;
+  if (ctx == nullptr || g_noalloc_ptr[dev] == nullptr || g_noalloc_ctx[dev] != static_cast<void*>(ctx)) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_ws);
+    e = cudaGetSymbolAddress(&p, g_noalloc_ws);  // makes the device's primary context current if needed
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static workspace)");
+    if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return fail(SOL_ECUDA, "no current CUDA context");
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = static_cast<void*>(ctx);
   }
   *out = g_noalloc_ptr[dev];
   return SOL_OK;
@@ -148,6 +185,11 @@ const char* sol_attn_status_string(sol_status s) {
 const char* sol_attn_last_error(void) { return g_last_error.c_str(); }
 
 void sol_attn_debug_drop_one_load(int mode) { g_drop_one_load = mode; }
+
+void sol_attn_debug_record_cta_times(unsigned long long* times, int capacity) {
+  g_cta_times = capacity > 0 ? times : nullptr;
+  g_cta_capacity = capacity > 0 ? capacity : 0;
+}
 
 sol_status sol_attn_pool(const void* K, const void* V, sol_dtype dt, int B, int H, int L, int d, int block_k,
                          float* kbar, float* vbar, void* kbar_lp, void* vbar_lp, void* stream) {
@@ -227,14 +269,18 @@ sol_status sol_attn_qknorm_rope_pool(const void* Q, const void* K, const void* V
 
 size_t sol_attn_fwd_workspace_bytes(int B, int H, int L, int block_q) {
   if (B < 1 || H < 1 || L < 1 || block_q < 1) return 0;
-  return ws_header_bytes(B, H) + ws_bits_bytes(B, H, L, block_q);
+  return ws_header_bytes(B, H) + ws_route_bytes(B, H, L, block_q);
 }
 
-sol_status sol_attn_fwd(const void* Q, const void* K, const void* V, const float* kbar, const float* vbar,
-                        const void* kbar_lp, const void* vbar_lp, const float* tau, sol_dtype dt, int B, int H, int L,
-                        int d, int block_q, int block_k, int n_force, void* O, uint8_t* kept_mask, float* density,
-                        void* workspace, size_t ws_bytes, void* stream) {
-  g_last_error.clear();
+}  // extern "C"
+
+namespace {
+
+// The forward of sol_attn_fwd; k_keep > 0 selects fixed-sparsity routing in the routing pass.
+sol_status fwd_impl(const void* Q, const void* K, const void* V, const float* kbar, const float* vbar,
+                    const void* kbar_lp, const void* vbar_lp, const float* tau, sol_dtype dt, int B, int H, int L,
+                    int d, int block_q, int block_k, int n_force, void* O, uint8_t* kept_mask, float* density,
+                    void* workspace, size_t ws_bytes, void* stream, int k_keep) {
   if (dt != SOL_F32 && dt != SOL_BF16) return fail(SOL_EINVAL, "unknown dtype %d", static_cast<int>(dt));
   if (!size_ok(B, 1 << 16) || !size_ok(H, 1 << 16) || !size_ok(L, 1 << 28) || !size_ok(d, 1 << 16) ||
       !size_ok(block_q, 1 << 20) || !size_ok(block_k, 1 << 20))
@@ -269,8 +315,9 @@ sol_status sol_attn_fwd(const void* Q, const void* K, const void* V, const float
   if (static_cast<long long>(B) * H > 65535) return fail(SOL_EUNSUPPORTED, "B*H must be <= 65535");
   const size_t need = ws_header_bytes(B, H);
   if (ws_bytes < need) return fail(SOL_EINVAL, "workspace too small (%zu < %zu bytes)", ws_bytes, need);
-  // a workspace that also holds the keep bits gets the separate routing pass (bf16 path)
-  const bool route_pass = bf16 && ws_bytes >= need + ws_bits_bytes(B, H, L, block_q);
+  // a workspace that also holds the keep bits and the query-block means gets the separate
+  // routing pass (bf16 path)
+  const bool route_pass = bf16 && ws_bytes >= need + ws_route_bytes(B, H, L, block_q);
 
   int sms = 0;
   sol_status st = current_device(&sms);
@@ -307,11 +354,19 @@ sol_status sol_attn_fwd(const void* Q, const void* K, const void* V, const float
   a.drop_one_load = 0;
   a.wait_limit_ns = 2000000000ull;
   a.route_bits = route_pass ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + need) : nullptr;
+  a.route_qbar = route_pass ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + need +
+                                                       ws_bits_bytes(B, H, L, block_q))
+                            : nullptr;
+  a.k_keep = k_keep;
 
   if (bf16) {
     a.drop_one_load = g_drop_one_load;
     if (g_drop_one_load) a.wait_limit_ns = 200000000ull;
     g_drop_one_load = 0;
+    a.cta_times = g_cta_times;
+    a.cta_capacity = g_cta_capacity;
+    g_cta_times = nullptr;
+    g_cta_capacity = 0;
     CUtensorMap maps[5];
     const int nkb_i = static_cast<int>(nkb);
     if ((st = make_map(&maps[0], Q, d, L, B * H)) != SOL_OK) return st;
@@ -332,6 +387,34 @@ sol_status sol_attn_fwd(const void* Q, const void* K, const void* V, const float
   return SOL_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+sol_status sol_attn_fwd(const void* Q, const void* K, const void* V, const float* kbar, const float* vbar,
+                        const void* kbar_lp, const void* vbar_lp, const float* tau, sol_dtype dt, int B, int H, int L,
+                        int d, int block_q, int block_k, int n_force, void* O, uint8_t* kept_mask, float* density,
+                        void* workspace, size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  return fwd_impl(Q, K, V, kbar, vbar, kbar_lp, vbar_lp, tau, dt, B, H, L, d, block_q, block_k, n_force, O, kept_mask,
+                  density, workspace, ws_bytes, stream, 0);
+}
+
+sol_status sol_attn_fwd_topk(const void* Q, const void* K, const void* V, const float* kbar, const void* kbar_lp,
+                             const void* vbar_lp, int k_keep, int B, int H, int L, int d, int n_force, void* O,
+                             uint8_t* kept_mask, float* density, void* workspace, size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  if (B < 1 || H < 1 || L < 1) return fail(SOL_EINVAL, "sizes must be positive (B=%d H=%d L=%d)", B, H, L);
+  if (H > sol::kMaxHeads) return fail(SOL_EUNSUPPORTED, "H=%d exceeds %d", H, sol::kMaxHeads);
+  const long long nkb = (static_cast<long long>(L) + 127) / 128;
+  if (k_keep < 1 || k_keep > nkb) return fail(SOL_EINVAL, "k_keep=%d must be in [1, N_kb=%lld]", k_keep, nkb);
+  if (workspace == nullptr || ws_bytes < sol_attn_fwd_workspace_bytes(B, H, L, 128))
+    return fail(SOL_EINVAL, "fixed-sparsity routing needs the full workspace (keep bits)");
+  float zeros[sol::kMaxHeads] = {};  // unused by the routing pass in this mode; valid thresholds
+  return fwd_impl(Q, K, V, kbar, nullptr, kbar_lp, vbar_lp, zeros, SOL_BF16, B, H, L, d, 128, 128, n_force, O,
+                  kept_mask, density, workspace, ws_bytes, stream, k_keep);
+}
+
 sol_status sol_attn_fwd_noalloc(const void* Q, const void* K, const void* V, const float* kbar, const float* vbar,
                                 const void* kbar_lp, const void* vbar_lp, const float* tau, sol_dtype dt, int B, int H,
                                 int L, int d, int block_q, int block_k, int n_force, void* O, uint8_t* kept_mask,
@@ -345,7 +428,7 @@ sol_status sol_attn_fwd_noalloc(const void* Q, const void* K, const void* V, con
   sol_status st = noalloc_workspace(&ws);
   if (st != SOL_OK) return st;
   // the array keeps the previous call's contents: clear all of it (counters and error word)
-  const size_t bytes = sizeof(uint32_t) * kNoAllocWords;
+  const size_t bytes = kNoAllocBytes;
   cudaError_t e = cudaMemsetAsync(ws, 0, bytes, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(static workspace)");
   return sol_attn_fwd(Q, K, V, kbar, vbar, kbar_lp, vbar_lp, tau, dt, B, H, L, d, block_q, block_k, n_force, O,
@@ -417,7 +500,7 @@ HostPlan host_plan(bool bf16, int B, int H, int L, int d, int block, int heads_p
   p.vbar_lp = off;
   off += pooled_lp;
   p.ws = off;
-  p.ws_bytes = round256(ws_header_bytes(1, p.c) + ws_bits_bytes(1, p.c, L, block));
+  p.ws_bytes = round256(ws_header_bytes(1, p.c) + ws_route_bytes(1, p.c, L, block));
   off += p.ws_bytes;
   p.dens = off;
   off += round256(static_cast<size_t>(B) * H * 4);

@@ -29,10 +29,12 @@ EXPORTED = (
     "sol_attn_fwd",
     "sol_attn_check_device_error",
     "sol_attn_debug_drop_one_load",
+    "sol_attn_debug_record_cta_times",
     "sol_attn_fwd_noalloc",
     "sol_attn_qknorm_rope_pool",
     "sol_attn_fwd_host_scratch_bytes",
     "sol_attn_fwd_host",
+    "sol_attn_fwd_topk",
 )
 
 
@@ -80,10 +82,15 @@ def load_library() -> ctypes.CDLL:
     lib.sol_attn_fwd_host.argtypes = [vp, vp, vp, vp, f32p, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp,
                                       ctypes.c_size_t, vp]
     lib.sol_attn_fwd_host.restype = i32
+    lib.sol_attn_fwd_topk.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp,
+                                      ctypes.c_size_t, vp]
+    lib.sol_attn_fwd_topk.restype = i32
     lib.sol_attn_check_device_error.argtypes = [vp, vp]
     lib.sol_attn_check_device_error.restype = i32
     lib.sol_attn_debug_drop_one_load.argtypes = [i32]
     lib.sol_attn_debug_drop_one_load.restype = None
+    lib.sol_attn_debug_record_cta_times.argtypes = [vp, i32]
+    lib.sol_attn_debug_record_cta_times.restype = None
     _lib = lib
     return lib
 
@@ -246,6 +253,27 @@ def sol_attn_fwd_noalloc(Q, K, V, kbar, vbar, kbar_lp, vbar_lp, tau: Sequence[fl
     return O
 
 
+def sol_attn_fwd_topk(Q, K, V, kbar, kbar_lp, vbar_lp, k_keep: int, n_force: int = 0, O=None, kept_mask=None,
+                      density=None, workspace=None, stream=None):
+    """Fused forward with fixed-sparsity routing: each query block keeps its k_keep highest-scoring
+    key blocks (bf16, blocks of 128). Returns O."""
+    _need_cuda("Q", Q, torch.bfloat16)
+    for n, t in (("K", K), ("V", V)):
+        _need_cuda(n, t, torch.bfloat16)
+    B, H, L, d = Q.shape
+    if K.shape != Q.shape or V.shape != Q.shape:
+        raise ValueError("Q, K and V must have the same shape [B, H, L, d]")
+    if O is None:
+        O = torch.empty_like(Q)
+    if workspace is None:
+        workspace = new_workspace(B, H, L, 128, Q.device)
+    st = load_library().sol_attn_fwd_topk(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(kbar), _ptr(kbar_lp), _ptr(vbar_lp), int(k_keep), B, H, L, d, int(n_force),
+        _ptr(O), _ptr(kept_mask), _ptr(density), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "sol_attn_fwd_topk")
+    return O
+
+
 def sol_attn_check_device_error(workspace: torch.Tensor, stream=None) -> None:
     """Synchronise and raise SolAttnError(SOL_ETIMEOUT) if a bounded device wait expired."""
     _check(load_library().sol_attn_check_device_error(_ptr(workspace), _stream(stream)),
@@ -254,6 +282,15 @@ def sol_attn_check_device_error(workspace: torch.Tensor, stream=None) -> None:
 
 def sol_attn_debug_drop_one_load(mode: int) -> None:
     load_library().sol_attn_debug_drop_one_load(int(mode))
+
+
+def sol_attn_debug_record_cta_times(times: torch.Tensor, capacity: int) -> None:
+    """Arm the next bf16 fused launch to write each CTA's (start, finish) globaltimer stamps into
+    `times` (int64 device tensor of at least 2 * capacity elements)."""
+    _need_cuda("times", times, torch.int64)
+    if times.numel() < 2 * capacity:
+        raise ValueError("times must hold 2 * capacity values")
+    load_library().sol_attn_debug_record_cta_times(_ptr(times), int(capacity))
 
 
 def sol_attn(Q, K, V, tau, block: int = 128, n_force: int = 0, want_mask: bool = False,

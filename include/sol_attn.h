@@ -106,17 +106,18 @@ sol_status sol_attn_qknorm_rope_pool(const void* Q, const void* K, const void* V
 
 /* Bytes of device workspace sol_attn_fwd needs for this problem. The workspace holds the
  * persistent scheduler's work counter, the per-(b,h) kept-block counters and the sticky device
- * error word (a header of 4 * (4 + B*H) bytes rounded up to 256), followed by the keep bits of the
- * routing pass: B*H*N_qb*ceil(N_kb/32) 32-bit words, rounded up to 256 bytes (1.8 MB for
- * B=1, H=40, L=75600, block 128). Zero it once after allocation; later calls keep it consistent. */
+ * error word (a header of 4 * (4 + B*H) bytes rounded up to 256), followed by the routing pass's
+ * keep bits, B*H*N_qb*ceil(N_kb/32) 32-bit words, and its query-block means, B*H*N_qb*128 floats,
+ * each rounded up to 256 bytes (1.8 MB + 12.1 MB for B=1, H=40, L=75600, block 128). Zero it once
+ * after allocation; later calls keep it consistent. */
 size_t sol_attn_fwd_workspace_bytes(int B, int H, int L, int block_q);
 
 /* The forward: routing, exact attention on kept blocks, skipped-block correction and the epilogue
  * (Sol-Attn project page, Abstract). For SOL_BF16 with a workspace of the full size returned above,
- * routing runs as its own pass first. That pass routes 4-16 query blocks of one head per CTA, so
- * each head's pooled keys are read once per group of query blocks instead of once per block. It
- * writes only the keep bits into the workspace, then the fused kernel turns them into its tile
- * lists. With a workspace that holds only the header, the fused kernel routes each query block
+ * routing runs as its own pass first. One kernel streams Q once and writes the query-block means
+ * q_bar into the workspace; a second routes 4-16 query blocks of one head per CTA, so each head's
+ * pooled keys are read once per group of query blocks instead of once per block, and writes only
+ * the keep bits into the workspace. The fused kernel then turns them into its tile lists. With a workspace that holds only the header, the fused kernel routes each query block
  * itself, with the same fp32 arithmetic in the same order, so both paths keep the same blocks.
  *
  *   Q, K, V     device, [B, H, L, d] in dtype `dt`
@@ -147,6 +148,18 @@ sol_status sol_attn_fwd(const void* Q, const void* K, const void* V, const float
                         int block_k, int n_force, void* O, uint8_t* kept_mask, float* density,
                         void* workspace, size_t ws_bytes, void* stream);
 
+/* The forward with fixed-sparsity routing: each query block keeps the k_keep key blocks with the
+ * highest proxy scores s_bar_ij (equal scores: the lower block index first), plus the first
+ * n_force blocks. The review page of the Sol Video Inference Engine paper names this kind of
+ * routing (PISA at sparsity 0.9) beside Sol-Attn's threshold. Exact tiles, correction and outputs
+ * are those of sol_attn_fwd. Only SOL_BF16 with blocks of 128 and d in {64, 128} is supported, and
+ * the workspace must have the full size of sol_attn_fwd_workspace_bytes (the routing pass writes
+ * the keep bits). 1 <= k_keep <= N_kb, else SOL_EINVAL. */
+sol_status sol_attn_fwd_topk(const void* Q, const void* K, const void* V, const float* kbar,
+                             const void* kbar_lp, const void* vbar_lp, int k_keep, int B, int H, int L,
+                             int d, int n_force, void* O, uint8_t* kept_mask, float* density,
+                             void* workspace, size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, then reads and clears the workspace's device error word. Returns
  * SOL_ETIMEOUT if any launch since the last check gave up on a bounded wait, after which that
  * launch's outputs are incomplete. Returns SOL_OK otherwise. */
@@ -159,21 +172,27 @@ sol_status sol_attn_check_device_error(void* workspace, void* stream);
  * already reserved the device memory and forbids foreign allocations; a plugin that must not
  * trigger the implicit device synchronisation cudaMalloc/cudaFree can cause on a latency-critical
  * path. Such callers cannot provide the workspace that sol_attn_fwd needs. This entry point takes
- * the same arguments minus the workspace. It uses a 16,400-byte array in the library's own device
+ * the same arguments minus the workspace. It uses a 16,640-byte array in the library's own device
  * memory instead: a file-scope static __device__ array, which every GPU that loads the library
  * holds until the process exits.
  *
- *   limit      B * H <= 4096 (the array holds the counters of at most 4096 heads); larger
+ *   limit      B * H <= 4096 (the array holds the workspace header of at most 4096 heads); larger
  *              problems return SOL_EUNSUPPORTED without launching anything.
- *   set-up     the first call on a device looks up the array's device address
- *              (cudaGetSymbolAddress) with that device current, and caches it. Make that first
- *              call before any stream capture.
+ *   routing    the array is passed to sol_attn_fwd as its workspace. When the routing pass's
+ *              keep bits and query-block means fit in what the header leaves free (see
+ *              sol_attn_fwd_workspace_bytes), the separate routing pass runs; otherwise the fused
+ *              kernel routes each unit itself. Both give the same results bit for bit.
+ *   set-up     the first call on a device (and the first after a cudaDeviceReset) looks up the
+ *              array's device address (cudaGetSymbolAddress) with that device current, and
+ *              caches it with the current context. Make that first call before any stream
+ *              capture.
  *   sharing    every call on a device shares the one array. Each call clears it on `stream`
  *              before launching, so calls on one stream are safe, but calls that overlap on the
  *              GPU (different streams, no ordering) race on it.
- *   errors     host-side errors as for sol_attn_fwd. The device error word of a bounded-wait
- *              expiry is kept in the shared array and is not readable through this ABI. Use
- *              sol_attn_fwd with a workspace when that status is needed.
+ *   errors     host-side errors as for sol_attn_fwd. A bounded-wait expiry on the device is
+ *              silent here: its error word lives in the shared array, is not readable through
+ *              this ABI, and the next call's clear erases it. Use sol_attn_fwd with a workspace
+ *              when that status is needed.
  * Calls no cudaMalloc, cudaFree or other allocating routine. */
 sol_status sol_attn_fwd_noalloc(const void* Q, const void* K, const void* V, const float* kbar,
                                 const float* vbar, const void* kbar_lp, const void* vbar_lp,
@@ -228,6 +247,13 @@ sol_status sol_attn_fwd_host(const void* Q, const void* K, const void* V, void* 
  * sol_attn_check_device_error then reports SOL_ETIMEOUT. The hook applies to one launch and
  * then resets to 0. The wait limit is about 0.2 s in that mode and about 2 s otherwise. */
 void sol_attn_debug_drop_one_load(int mode);
+
+/* Measurement hook for the persistent scheduler's load balance. The next sol_attn_fwd launch of
+ * the SOL_BF16 fused kernel writes, for each CTA c < capacity, its start and finish time in
+ * nanoseconds (the GPU's global timer) to times[2c] and times[2c + 1]. `times` is device memory
+ * of 2 * capacity 64-bit words, owned by the caller. The hook applies to one launch and then
+ * resets; capacity <= 0 disarms it. */
+void sol_attn_debug_record_cta_times(unsigned long long* times, int capacity);
 
 #ifdef __cplusplus
 }

@@ -47,9 +47,11 @@ def test_workspace_size(lib):
     assert n % 256 == 0 and n >= 4 * (4 + 64)
     assert sa.sol_attn_fwd_workspace_bytes(0, 1, 1, 1) == 0
     # header (error, where, counter, done, 40 per-head counts) + keep bits 40 x 591 x ceil(591/32) words
+    # + query-block means 40 x 591 x 128 floats
     header = ((4 + 40) * 4 + 255) // 256 * 256
     bits = -(-(40 * 591 * 19 * 4) // 256) * 256
-    assert sa.sol_attn_fwd_workspace_bytes(1, 40, 75600, 128) == header + bits
+    qbar = -(-(40 * 591 * 128 * 4) // 256) * 256
+    assert sa.sol_attn_fwd_workspace_bytes(1, 40, 75600, 128) == header + bits + qbar
 
 
 # fake, 16-byte aligned device addresses: validation must reject before any of them is used
@@ -136,11 +138,12 @@ def test_host_entry_scratch_size(lib):
     # of a 2-head call and 40 density words, each rounded up to 256 bytes
     r = lambda x: -(-x // 256) * 256  # noqa: E731
     L, d, c, H, nkb = 75600, 128, 2, 40, 591
-    ws = r(r((4 + c) * 4) + r(c * nkb * 19 * 4))
+    ws = r(r((4 + c) * 4) + r(c * nkb * 19 * 4) + r(c * nkb * 128 * 4))  # header, keep bits, q_bar
     want = 8 * r(c * L * d * 2) + 2 * r(c * nkb * d * 4) + 2 * r(c * nkb * d * 2) + ws + r(H * 4)
     assert lib.sol_attn_fwd_host_scratch_bytes(sa.SOL_BF16, 1, H, L, d, 128, c) == want
     # fp32: 4-byte elements, no bf16 mirrors
-    want32 = 8 * r(c * 1000 * 64 * 4) + 2 * r(c * 16 * 64 * 4) + r(r((4 + c) * 4) + r(c * 16 * 1 * 4)) + r(3 * 4)
+    want32 = (8 * r(c * 1000 * 64 * 4) + 2 * r(c * 16 * 64 * 4) +
+              r(r((4 + c) * 4) + r(c * 16 * 1 * 4) + r(c * 16 * 128 * 4)) + r(3 * 4))
     assert lib.sol_attn_fwd_host_scratch_bytes(sa.SOL_F32, 1, 3, 1000, 64, 64, c) == want32
     # more heads per chunk than heads: one chunk of H heads
     assert (lib.sol_attn_fwd_host_scratch_bytes(sa.SOL_BF16, 2, 3, 1000, 64, 128, 99) ==
@@ -181,3 +184,16 @@ def test_host_binding_rejects_non_host_tensors(lib):
     x = torch.zeros(1, 1, 8, 64)
     with pytest.raises(ValueError):
         sa.sol_attn_fwd_host(x, x, torch.zeros(1, 1, 8, 32), [1.0])
+
+
+def test_topk_entry_rejects_invalid_arguments(lib):
+    def call(k=3, L=1000, ws=1 << 30, workspace=P[8], B=1, H=2):
+        return lib.sol_attn_fwd_topk(P[0], P[1], P[2], P[3], P[4], P[5], k, B, H, L, 128, 0, P[7], None, None,
+                                     workspace, ws, None)
+    assert call(k=0) == sa.SOL_EINVAL
+    assert call(k=9) == sa.SOL_EINVAL  # N_kb = 8
+    assert call(ws=16) == sa.SOL_EINVAL
+    assert "full workspace" in lib.sol_attn_last_error().decode()
+    assert call(workspace=None) == sa.SOL_EINVAL
+    assert call(L=0) == sa.SOL_EINVAL
+    assert call(H=300) == sa.SOL_EUNSUPPORTED

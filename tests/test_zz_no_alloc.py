@@ -44,13 +44,17 @@ def _inputs(B, H, L, d, dtype, seed):
     return [torch.from_numpy(np.asarray(a, dtype=np.float32)).to(dtype).cuda() for a in arrs]
 
 
-@pytest.mark.parametrize("dtype,L,d,block,tau", [
-    (torch.bfloat16, 3000, 128, 128, [0.0, 0.7, 2.5, math.inf]),
-    (torch.bfloat16, 1500, 64, 128, [0.4, 1.0, 1.5, 3.0]),
-    (torch.float32, 700, 64, 64, [0.3, 1.2, 2.0, math.inf]),
+@pytest.mark.parametrize("B,H,dtype,L,d,block,tau", [
+    (1, 4, torch.bfloat16, 3000, 128, 128, [0.0, 0.7, 2.5, math.inf]),
+    (1, 4, torch.bfloat16, 1500, 64, 128, [0.4, 1.0, 1.5, 3.0]),
+    (1, 4, torch.float32, 700, 64, 64, [0.3, 1.2, 2.0, math.inf]),
+    # 200 key blocks: the keep bits (4 heads x 200 x 7 words) do not fit beside the header, so
+    # the fused kernel routes in-kernel on this entry point
+    (1, 4, torch.bfloat16, 25_600, 128, 128, [0.3, 0.8, 1.5, 4.0]),
+    # the limit: B*H = 4096 heads fill the array's header exactly
+    (16, 256, torch.bfloat16, 130, 64, 128, [0.5] * 256),
 ])
-def test_noalloc_matches_workspace_entry_point_twice(dtype, L, d, block, tau):
-    B, H = 1, 4
+def test_noalloc_matches_workspace_entry_point_twice(B, H, dtype, L, d, block, tau):
     Q, K, V = _inputs(B, H, L, d, dtype, seed=L + d)
     kbar, vbar, klp, vlp = sa.sol_attn_pool(K, V, block)
     nb = -(-L // block)
