@@ -21,7 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libsolattn.so")
 
-SOURCES = ["pool.cu", "rope_pool.cu", "route.cu", "fwd_simt.cu", "fwd_tc.cu", "sol_attn_api.cu"]
+SOURCES = ["pool.cu", "rope_pool.cu", "route.cu", "quant.cu", "fwd_simt.cu", "fwd_tc.cu", "sol_attn_api.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", "-I", CSRC, "-I", INCLUDE]

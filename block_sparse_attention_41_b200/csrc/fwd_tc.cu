@@ -790,6 +790,7 @@ cudaError_t launch_tc_t(const FwdArgs& a, const CUtensorMap* maps, cudaStream_t 
 }  // namespace
 
 cudaError_t launch_fwd_tc(const FwdArgs& a, const CUtensorMap* maps, cudaStream_t stream) {
+  if (a.qk8 != nullptr) return cudaErrorNotSupported;
   if (a.d == 64) return launch_tc_t<64>(a, maps, stream);
   if (a.d == 128) return launch_tc_t<128>(a, maps, stream);
   return cudaErrorInvalidValue;

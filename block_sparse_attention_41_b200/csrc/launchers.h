@@ -8,6 +8,16 @@
 
 namespace sol {
 
+// 8-bit QK^T operands of the forward (sol_attn_quantize_qk8): codes and per-tile scales
+struct Qk8Operands {
+  const int8_t* q8;        // [BH, L, d]
+  const int8_t* k8;        // [BH, L, d], K - mu
+  const int8_t* kb8;       // [BH, N_kb, d], k_bar - mu
+  const float* q_scale;    // [BH, N_qb]
+  const float* k_scale;    // [BH, N_kb]
+  const float* kb_scale;   // [BH, ceil(N_kb / 128)]
+};
+
 struct FwdArgs {
   const void* Q;
   const void* K;
@@ -33,6 +43,7 @@ struct FwdArgs {
   int k_keep = 0;          // routing pass: 0 = threshold max - tau; k > 0 = the k highest scores
   unsigned long long* cta_times = nullptr;  // measurement hook: [2 * cta_capacity] start/finish ns
   int cta_capacity = 0;
+  const Qk8Operands* qk8 = nullptr;  // bf16 path: int8 Q, K and pooled keys for QK^T, or null
 };
 
 cudaError_t launch_pool(const void* K, const void* V, bool bf16, int BH, int L, int d, int block,
@@ -55,6 +66,24 @@ struct RopePoolArgs {
   void* vbar_lp;
   int BH, L, d, block;
 };
+
+struct QuantArgs {
+  const void* Q;       // bf16 [BH, L, d]
+  const void* K;       // bf16 [BH, L, d]
+  const float* kbar;   // fp32 [BH, N_kb, d] from the pooling pass
+  float* mu;           // out: fp32 [BH, d] mean key
+  int8_t* q8;          // out: int8 [BH, L, d]
+  int8_t* k8;          // out: int8 [BH, L, d] codes of K - mu
+  int8_t* kb8;         // out: int8 [BH, N_kb, d] codes of k_bar - mu
+  float* q_scale;      // out: [BH, N_qb]
+  float* k_scale;      // out: [BH, N_kb]
+  float* kb_scale;     // out: [BH, ceil(N_kb / 128)]
+  int BH, L, d;
+};
+
+// bf16, d in {64, 128}, blocks of 128: the mean key, then int8 codes and tile scales of Q, K - mu
+// and k_bar - mu.
+cudaError_t launch_quant_qk8(const QuantArgs& a, cudaStream_t stream);
 
 // bf16, d in {64, 128}: QK RMS norm + rotary embedding + K/V block pooling in one pass.
 cudaError_t launch_qknorm_rope_pool(const RopePoolArgs& a, cudaStream_t stream);

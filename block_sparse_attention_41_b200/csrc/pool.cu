@@ -4,8 +4,9 @@
 //
 // HBM-bound: every K and V element is read exactly once with 16-byte vector loads; the output
 // is 1/block of the input. One CTA pools one key block of one tensor (K or V) of one head.
-// Each thread owns a 16-byte column slice and sums every `rows_per_pass`-th row in fp32, so
-// the summation order is fixed and the result is deterministic.
+// Each thread owns a 16-byte column slice and sums every `rows_per_pass`-th row in fp32. The row
+// groups that share a warp are then added with warp shuffles, and the warps' sums through shared
+// memory, always in the same order, so the result is deterministic.
 #include <cuda_bf16.h>
 
 #include "device_common.cuh"
@@ -45,7 +46,8 @@ __global__ void __launch_bounds__(kPoolThreads)
                     float* __restrict__ kbar, float* __restrict__ vbar, __nv_bfloat16* __restrict__ kbar_lp,
                     __nv_bfloat16* __restrict__ vbar_lp) {
   constexpr int VEC = 16 / sizeof(T);
-  __shared__ float partial[kPoolThreads * VEC];
+  constexpr int kWarps = kPoolThreads / 32;
+  __shared__ float partial[kWarps][256];  // d <= 256 (bf16) or 128 (fp32)
 
   const int j = blockIdx.x;
   const int bh = blockIdx.y;
@@ -63,7 +65,7 @@ __global__ void __launch_bounds__(kPoolThreads)
 #pragma unroll
   for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
 
-  if (r0 < rows_per_pass) {
+  {
     const uint4* base = reinterpret_cast<const uint4*>(src) + c;
     const size_t row_stride = static_cast<size_t>(lanes_per_row);  // in uint4
     int r = r0;
@@ -79,17 +81,25 @@ __global__ void __launch_bounds__(kPoolThreads)
       add_vec<T>(acc, x3);
     }
     for (; r < n; r += rows_per_pass) add_vec<T>(acc, __ldg(base + static_cast<size_t>(r) * row_stride));
+  }
+  // the row groups inside a warp sit lanes_per_row lanes apart (lanes_per_row = d / VEC divides 32)
+  for (int o = lanes_per_row; o < 32; o <<= 1) {
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) partial[r0 * d + c * VEC + v] = acc[v];
+    for (int v = 0; v < VEC; ++v) acc[v] += __shfl_xor_sync(0xffffffffu, acc[v], o);
+  }
+  const int warp = tid >> 5, lane = tid & 31;
+  if (lane < lanes_per_row) {
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) partial[warp][c * VEC + v] = acc[v];
   }
   __syncthreads();
 
   float* out = (is_v ? vbar : kbar) + (static_cast<size_t>(bh) * nkb + j) * d;
   __nv_bfloat16* out_lp = is_v ? vbar_lp : kbar_lp;
-  const int used_rows = min(rows_per_pass, n);
   for (int col = tid; col < d; col += kPoolThreads) {
     float s = 0.f;
-    for (int r = 0; r < used_rows; ++r) s += partial[r * d + col];
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) s += partial[w][col];
     const float mean = s / static_cast<float>(n);
     out[col] = mean;
     if (out_lp != nullptr) out_lp[(static_cast<size_t>(bh) * nkb + j) * d + col] = __float2bfloat16_rn(mean);

@@ -70,16 +70,18 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D bf16 view [BH][rows][d] with 64 x 128 x 1 boxes and 128-byte swizzle. Rows past `rows`
-// (a ragged last block) are zero-filled by the copy engine.
-sol_status make_map(CUtensorMap* m, const void* base, int d, int rows, int BH) {
+// 3-D view [BH][rows][d] with 128-byte-wide x 128 x 1 boxes (64 bf16 or 128 int8 values) and
+// 128-byte swizzle. Rows past `rows` (a ragged last block) are zero-filled by the copy engine.
+sol_status make_map(CUtensorMap* m, const void* base, int d, int rows, int BH, bool int8 = false) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return fail(SOL_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t es = int8 ? 1 : 2;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(rows) * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * es, static_cast<cuuint64_t>(rows) * d * es};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / es), 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = fn(m, int8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(SOL_ECUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
@@ -210,8 +212,11 @@ sol_status sol_attn_pool(const void* K, const void* V, sol_dtype dt, int B, int 
     return fail(SOL_EINVAL, "kbar_lp and vbar_lp must be NULL for fp32 inputs");
   if (bf16 && (!aligned16(kbar_lp) || !aligned16(vbar_lp)))
     return fail(SOL_EINVAL, "device pointers must be 16-byte aligned");
-  if (d > 512 || d % (bf16 ? 8 : 4) != 0)
-    return fail(SOL_EUNSUPPORTED, "pool needs d <= 512 and d %% %d == 0 (d=%d)", bf16 ? 8 : 4, d);
+  // a row is d / VEC 16-byte vectors (VEC = 8 bf16 or 4 fp32 values); the pool kernel needs that
+  // count to be a power of two of at most 32, so the row groups of a warp reduce by shuffles
+  const int vecs = d / (bf16 ? 8 : 4);
+  if (d % (bf16 ? 8 : 4) != 0 || vecs > 32 || (vecs & (vecs - 1)) != 0)
+    return fail(SOL_EUNSUPPORTED, "pool needs d / %d to be a power of two <= 32 (d=%d)", bf16 ? 8 : 4, d);
   if (block_k > 4096) return fail(SOL_EUNSUPPORTED, "pool needs block_k <= 4096");
   if ((L + block_k - 1) / block_k > 0x7fffffff / 1) return fail(SOL_EUNSUPPORTED, "too many blocks");
   int sms = 0;
@@ -267,6 +272,43 @@ sol_status sol_attn_qknorm_rope_pool(const void* Q, const void* K, const void* V
   return SOL_OK;
 }
 
+sol_status sol_attn_quantize_qk8(const void* Q, const void* K, const float* kbar, int B, int H, int L, int d,
+                                 int8_t* q8, int8_t* k8, int8_t* kbar8, float* q_scale, float* k_scale,
+                                 float* kbar_scale, float* mu, void* stream) {
+  g_last_error.clear();
+  if (!size_ok(B, 1 << 16) || !size_ok(H, 1 << 16) || !size_ok(L, 1 << 28) || !size_ok(d, 1 << 16))
+    return fail(SOL_EINVAL, "sizes must be positive (B=%d H=%d L=%d d=%d)", B, H, L, d);
+  const void* ptrs[] = {Q, K, kbar, q8, k8, kbar8, q_scale, k_scale, kbar_scale, mu};
+  for (const void* ptr : ptrs) {
+    if (ptr == nullptr) return fail(SOL_EINVAL, "every pointer argument must be non-null");
+    if (!aligned16(ptr)) return fail(SOL_EINVAL, "device pointers must be 16-byte aligned");
+  }
+  if (d != 64 && d != 128) return fail(SOL_EUNSUPPORTED, "8-bit operands need d in {64, 128} (d=%d)", d);
+  if (static_cast<long long>(B) * H > 65535) return fail(SOL_EUNSUPPORTED, "B*H must be <= 65535");
+  const long long nkb = (static_cast<long long>(L) + 127) / 128;
+  if (nkb > sol::kMaxKeyBlocks) return fail(SOL_EUNSUPPORTED, "N_kb=%lld exceeds %d", nkb, sol::kMaxKeyBlocks);
+  int sms = 0;
+  sol_status st = current_device(&sms);
+  if (st != SOL_OK) return st;
+  sol::QuantArgs a;
+  a.Q = Q;
+  a.K = K;
+  a.kbar = kbar;
+  a.mu = mu;
+  a.q8 = q8;
+  a.k8 = k8;
+  a.kb8 = kbar8;
+  a.q_scale = q_scale;
+  a.k_scale = k_scale;
+  a.kb_scale = kbar_scale;
+  a.BH = B * H;
+  a.L = L;
+  a.d = d;
+  cudaError_t e = sol::launch_quant_qk8(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "8-bit quantization launch");
+  return SOL_OK;
+}
+
 size_t sol_attn_fwd_workspace_bytes(int B, int H, int L, int block_q) {
   if (B < 1 || H < 1 || L < 1 || block_q < 1) return 0;
   return ws_header_bytes(B, H) + ws_route_bytes(B, H, L, block_q);
@@ -280,7 +322,8 @@ namespace {
 sol_status fwd_impl(const void* Q, const void* K, const void* V, const float* kbar, const float* vbar,
                     const void* kbar_lp, const void* vbar_lp, const float* tau, sol_dtype dt, int B, int H, int L,
                     int d, int block_q, int block_k, int n_force, void* O, uint8_t* kept_mask, float* density,
-                    void* workspace, size_t ws_bytes, void* stream, int k_keep) {
+                    void* workspace, size_t ws_bytes, void* stream, int k_keep,
+                    const sol::Qk8Operands* qk8 = nullptr) {
   if (dt != SOL_F32 && dt != SOL_BF16) return fail(SOL_EINVAL, "unknown dtype %d", static_cast<int>(dt));
   if (!size_ok(B, 1 << 16) || !size_ok(H, 1 << 16) || !size_ok(L, 1 << 28) || !size_ok(d, 1 << 16) ||
       !size_ok(block_q, 1 << 20) || !size_ok(block_k, 1 << 20))
@@ -369,11 +412,13 @@ sol_status fwd_impl(const void* Q, const void* K, const void* V, const float* kb
     g_cta_capacity = 0;
     CUtensorMap maps[5];
     const int nkb_i = static_cast<int>(nkb);
-    if ((st = make_map(&maps[0], Q, d, L, B * H)) != SOL_OK) return st;
-    if ((st = make_map(&maps[1], K, d, L, B * H)) != SOL_OK) return st;
+    const bool i8 = qk8 != nullptr;  // Q, K and the pooled keys as int8 codes
+    if ((st = make_map(&maps[0], i8 ? qk8->q8 : Q, d, L, B * H, i8)) != SOL_OK) return st;
+    if ((st = make_map(&maps[1], i8 ? qk8->k8 : K, d, L, B * H, i8)) != SOL_OK) return st;
     if ((st = make_map(&maps[2], V, d, L, B * H)) != SOL_OK) return st;
-    if ((st = make_map(&maps[3], kbar_lp, d, nkb_i, B * H)) != SOL_OK) return st;
+    if ((st = make_map(&maps[3], i8 ? qk8->kb8 : kbar_lp, d, nkb_i, B * H, i8)) != SOL_OK) return st;
     if ((st = make_map(&maps[4], vbar_lp, d, nkb_i, B * H)) != SOL_OK) return st;
+    a.qk8 = qk8;
     if (route_pass) {
       e = sol::launch_route(a, s);
       if (e != cudaSuccess) return cuda_fail(e, "routing launch");
@@ -413,6 +458,27 @@ sol_status sol_attn_fwd_topk(const void* Q, const void* K, const void* V, const 
   float zeros[sol::kMaxHeads] = {};  // unused by the routing pass in this mode; valid thresholds
   return fwd_impl(Q, K, V, kbar, nullptr, kbar_lp, vbar_lp, zeros, SOL_BF16, B, H, L, d, 128, 128, n_force, O,
                   kept_mask, density, workspace, ws_bytes, stream, k_keep);
+}
+
+sol_status sol_attn_fwd_qk8(const void* Q, const int8_t* q8, const int8_t* k8, const int8_t* kbar8,
+                            const float* q_scale, const float* k_scale, const float* kbar_scale, const void* V,
+                            const float* kbar, const void* vbar_lp, const float* tau, int B, int H, int L, int d,
+                            int n_force, void* O, uint8_t* kept_mask, float* density, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  if (B < 1 || H < 1 || L < 1) return fail(SOL_EINVAL, "sizes must be positive (B=%d H=%d L=%d)", B, H, L);
+  const void* ptrs[] = {q8, k8, kbar8, q_scale, k_scale, kbar_scale};
+  for (const void* ptr : ptrs) {
+    if (ptr == nullptr) return fail(SOL_EINVAL, "every 8-bit operand and scale must be non-null");
+    if (!aligned16(ptr)) return fail(SOL_EINVAL, "device pointers must be 16-byte aligned");
+  }
+  if (d != 128) return fail(SOL_EUNSUPPORTED, "8-bit QK^T needs d = 128 (d=%d)", d);
+  if (workspace == nullptr || ws_bytes < sol_attn_fwd_workspace_bytes(B, H, L, 128))
+    return fail(SOL_EINVAL, "8-bit QK^T needs the full workspace (its routing pass reads the bf16 Q)");
+  sol::Qk8Operands ops{q8, k8, kbar8, q_scale, k_scale, kbar_scale};
+  // K is not read on this path; k8 stands in for it in the argument checks
+  return fwd_impl(Q, k8, V, kbar, nullptr, vbar_lp, vbar_lp, tau, SOL_BF16, B, H, L, d, 128, 128, n_force, O,
+                  kept_mask, density, workspace, ws_bytes, stream, 0, &ops);
 }
 
 sol_status sol_attn_fwd_noalloc(const void* Q, const void* K, const void* V, const float* kbar, const float* vbar,

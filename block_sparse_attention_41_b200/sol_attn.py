@@ -35,6 +35,8 @@ EXPORTED = (
     "sol_attn_fwd_host_scratch_bytes",
     "sol_attn_fwd_host",
     "sol_attn_fwd_topk",
+    "sol_attn_quantize_qk8",
+    "sol_attn_fwd_qk8",
 )
 
 
@@ -77,6 +79,11 @@ def load_library() -> ctypes.CDLL:
     lib.sol_attn_qknorm_rope_pool.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, i32, i32, i32, i32,
                                               vp, vp, vp, vp, vp, vp, vp]
     lib.sol_attn_qknorm_rope_pool.restype = i32
+    lib.sol_attn_quantize_qk8.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.sol_attn_quantize_qk8.restype = i32
+    lib.sol_attn_fwd_qk8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, f32p, i32, i32, i32, i32, i32, vp, vp,
+                                     vp, vp, ctypes.c_size_t, vp]
+    lib.sol_attn_fwd_qk8.restype = i32
     lib.sol_attn_fwd_host_scratch_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32]
     lib.sol_attn_fwd_host_scratch_bytes.restype = ctypes.c_size_t
     lib.sol_attn_fwd_host.argtypes = [vp, vp, vp, vp, f32p, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp,
@@ -188,6 +195,58 @@ def sol_attn_qknorm_rope_pool(Q, K, V, gain_q, gain_k, rope_cos, rope_sin, block
         _stream(stream))
     _check(st, "sol_attn_qknorm_rope_pool")
     return Q_out, K_out, kbar, vbar, kbar_lp, vbar_lp
+
+
+def sol_attn_quantize_qk8(Q, K, kbar, stream=None):
+    """8-bit QK^T operands (blocks of 128): returns (q8, k8, kbar8, q_scale, k_scale, kbar_scale, mu),
+    the int8 codes of Q, K - mu and kbar - mu with one scale per 128-row tile, and the mean key mu."""
+    for n, t in (("Q", Q), ("K", K)):
+        _need_cuda(n, t, torch.bfloat16)
+    _need_cuda("kbar", kbar, torch.float32)
+    B, H, L, d = Q.shape
+    nkb = -(-L // 128)
+    if K.shape != Q.shape or tuple(kbar.shape) != (B, H, nkb, d):
+        raise ValueError("Q, K must be [B, H, L, d] and kbar [B, H, ceil(L/128), d]")
+    dev = Q.device
+    q8 = torch.empty((B, H, L, d), dtype=torch.int8, device=dev)
+    k8 = torch.empty_like(q8)
+    kbar8 = torch.empty((B, H, nkb, d), dtype=torch.int8, device=dev)
+    q_scale = torch.empty((B, H, nkb), dtype=torch.float32, device=dev)
+    k_scale = torch.empty_like(q_scale)
+    kbar_scale = torch.empty((B, H, -(-nkb // 128)), dtype=torch.float32, device=dev)
+    mu = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+    st = load_library().sol_attn_quantize_qk8(
+        _ptr(Q), _ptr(K), _ptr(kbar), B, H, L, d, _ptr(q8), _ptr(k8), _ptr(kbar8), _ptr(q_scale), _ptr(k_scale),
+        _ptr(kbar_scale), _ptr(mu), _stream(stream))
+    _check(st, "sol_attn_quantize_qk8")
+    return q8, k8, kbar8, q_scale, k_scale, kbar_scale, mu
+
+
+def sol_attn_fwd_qk8(Q, q8, k8, kbar8, q_scale, k_scale, kbar_scale, V, kbar, vbar_lp, tau: Sequence[float],
+                     n_force: int = 0, O=None, kept_mask=None, density=None, workspace=None, stream=None):
+    """The forward with 8-bit QK^T from the operands of sol_attn_quantize_qk8 (d = 128). Returns O."""
+    _need_cuda("Q", Q, torch.bfloat16)
+    _need_cuda("V", V, torch.bfloat16)
+    B, H, L, d = Q.shape
+    for n, t in (("q8", q8), ("k8", k8), ("kbar8", kbar8)):
+        _need_cuda(n, t, torch.int8)
+    for n, t in (("q_scale", q_scale), ("k_scale", k_scale), ("kbar_scale", kbar_scale), ("kbar", kbar)):
+        _need_cuda(n, t, torch.float32)
+    _need_cuda("vbar_lp", vbar_lp, torch.bfloat16)
+    tau = [float(x) for x in tau]
+    if len(tau) != H:
+        raise ValueError(f"tau must hold H={H} values")
+    if O is None:
+        O = torch.empty_like(Q)
+    if workspace is None:
+        workspace = new_workspace(B, H, L, 128, Q.device)
+    tau_c = (ctypes.c_float * H)(*tau)
+    st = load_library().sol_attn_fwd_qk8(
+        _ptr(Q), _ptr(q8), _ptr(k8), _ptr(kbar8), _ptr(q_scale), _ptr(k_scale), _ptr(kbar_scale), _ptr(V), _ptr(kbar),
+        _ptr(vbar_lp), tau_c, B, H, L, d, int(n_force), _ptr(O), _ptr(kept_mask), _ptr(density), _ptr(workspace),
+        workspace.numel(), _stream(stream))
+    _check(st, "sol_attn_fwd_qk8")
+    return O
 
 
 def sol_attn_fwd_workspace_bytes(B: int, H: int, L: int, block_q: int) -> int:

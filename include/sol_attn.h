@@ -72,7 +72,8 @@ const char* sol_attn_last_error(void);
  *   kbar_lp,  device, bfloat16 [B, H, N_kb, d]: the same means rounded to bf16 (nearest even),
  *   vbar_lp   the operands of the tensor-core correction tiles. Required when dt == SOL_BF16,
  *             must be NULL when dt == SOL_F32.
- * Supported: SOL_BF16 with d % 8 == 0, SOL_F32 with d % 4 == 0, d <= 512, 1 <= block_k <= 4096.
+ * Supported: d / 8 (SOL_BF16) or d / 4 (SOL_F32) a power of two <= 32, i.e. d in {8, ..., 256} or
+ * {4, ..., 128}; 1 <= block_k <= 4096.
  */
 sol_status sol_attn_pool(const void* K, const void* V, sol_dtype dt, int B, int H, int L, int d,
                          int block_k, float* kbar, float* vbar, void* kbar_lp, void* vbar_lp,
@@ -103,6 +104,24 @@ sol_status sol_attn_qknorm_rope_pool(const void* Q, const void* K, const void* V
                                      float eps, int B, int H, int L, int d, int block_k, void* Q_out,
                                      void* K_out, float* kbar, float* vbar, void* kbar_lp, void* vbar_lp,
                                      void* stream);
+
+/* 8-bit operands of QK^T for sol_attn_fwd_qk8 (NEXT-2: the review page of the Sol Video Inference
+ * Engine paper lists SageAttention's 8-bit attention with outlier smoothing; the Sol-Engine README
+ * news reports fused 8-bit compute). From Q, K (bf16 [B, H, L, d]) and the fp32 pooled keys kbar
+ * of sol_attn_pool, with blocks of 128:
+ *   mu          device, out, float32 [B, H, d]: the head's mean key, sum_j n_j kbar_j / L
+ *   q8          device, out, int8 [B, H, L, d]: Q, one scale per 128-row query block
+ *   k8          device, out, int8 [B, H, L, d]: K - mu, one scale per key block
+ *   kbar8       device, out, int8 [B, H, N_kb, d]: kbar - mu, one scale per chunk of 128 pooled keys
+ *   q_scale     device, out, float32 [B, H, N_qb];  k_scale [B, H, N_kb];  kbar_scale
+ *               [B, H, ceil(N_kb / 128)]: amax / 127 of each tile (1 for an all-zero tile)
+ * A code is the fp32 round-to-nearest-even of x * 127 / amax, clamped to [-127, 127]. Subtracting
+ * mu shifts every logit of a query row by the same amount, so in exact arithmetic it changes
+ * nothing; it keeps a common key offset out of the 8-bit range (SageAttention's smoothing).
+ * d in {64, 128}, N_kb <= 4096, all pointers 16-byte aligned. Asynchronous on `stream`. */
+sol_status sol_attn_quantize_qk8(const void* Q, const void* K, const float* kbar, int B, int H, int L,
+                                 int d, int8_t* q8, int8_t* k8, int8_t* kbar8, float* q_scale,
+                                 float* k_scale, float* kbar_scale, float* mu, void* stream);
 
 /* Bytes of device workspace sol_attn_fwd needs for this problem. The workspace holds the
  * persistent scheduler's work counter, the per-(b,h) kept-block counters and the sticky device
@@ -159,6 +178,19 @@ sol_status sol_attn_fwd_topk(const void* Q, const void* K, const void* V, const 
                              const void* kbar_lp, const void* vbar_lp, int k_keep, int B, int H, int L,
                              int d, int n_force, void* O, uint8_t* kept_mask, float* density,
                              void* workspace, size_t ws_bytes, void* stream);
+
+/* The forward with 8-bit QK^T (NEXT-2): the exact tiles' and the correction's scores come from the
+ * int8 codes of sol_attn_quantize_qk8 (tcgen05 kind::i8, int32 accumulation), scaled by
+ * q_scale * k_scale (or kbar_scale for a pooled tile) in the softmax; P and V stay bf16. Routing
+ * is unchanged: the routing pass reads the bf16 Q and the fp32 pooled keys kbar, so the kept
+ * blocks are those of sol_attn_fwd. vbar_lp is the bf16 pooled V of sol_attn_pool. SOL_BF16 only,
+ * d = 128, blocks of 128, and the workspace must have the full size of
+ * sol_attn_fwd_workspace_bytes. Other arguments, limits and errors as for sol_attn_fwd. */
+sol_status sol_attn_fwd_qk8(const void* Q, const int8_t* q8, const int8_t* k8, const int8_t* kbar8,
+                            const float* q_scale, const float* k_scale, const float* kbar_scale,
+                            const void* V, const float* kbar, const void* vbar_lp, const float* tau,
+                            int B, int H, int L, int d, int n_force, void* O, uint8_t* kept_mask,
+                            float* density, void* workspace, size_t ws_bytes, void* stream);
 
 /* Synchronises `stream`, then reads and clears the workspace's device error word. Returns
  * SOL_ETIMEOUT if any launch since the last check gave up on a bounded wait, after which that

@@ -13,6 +13,15 @@ complete after random delays. A run fails on:
 
 Barrier semantics: a barrier of count c completes a phase after c arrivals; a wait for phase k
 (parity k & 1) passes once k + 1 phases have completed.
+
+Three schedules are modelled. "split" (the kernel's): both softmax groups work on every tile,
+each on half of its key columns, one thread issues every QK^T and one PV issuer per group
+consumes every tile. "alternate": softmax group g takes the tiles t of each unit with
+t & 1 == g (so the split does not depend on what the CTA ran before), owns S buffer g and its
+own PV issuer, and rescales its accumulator without waiting, because its previous PV completed
+before the QK^T that filled its S buffer was issued. "group_issuers": as "alternate", with one
+thread per group issuing both the group's QK^T and its PV. The last two were measured slower
+than "split" on the GPU; the model keeps their protocols checked.
 """
 from __future__ import annotations
 
@@ -33,17 +42,24 @@ class Bar:
 class Protocol:
     """One CTA running `plan` (tiles per unit) with the kernel's K and V ring depths."""
 
-    def __init__(self, plan, seed, nk=3, nv=2, mutation=None, route_in_kernel=False):
+    def __init__(self, plan, seed, nk=3, nv=2, mutation=None, route_in_kernel=False, schedule="split"):
         self.plan, self.nk, self.nv, self.mut = plan, nk, nv, mutation
         self.route_in_kernel = route_in_kernel  # no keep bits given: the softmax warps route from the Q tile
+        self.alt = schedule in ("alternate", "group_issuers")
+        self.group_issuers = schedule == "group_issuers"
         self.rng = random.Random(seed)
         self.now, self.seq, self.events = 0, 0, []
-        pv_count = 1 if mutation == "pvdone_count_1" else 2
+        if self.alt:  # one PV per tile: the owning group's
+            pv_count = 2 if mutation == "alt_pvdone_count_2" else 1
+            v_count = 1
+        else:
+            pv_count = 1 if mutation == "pvdone_count_1" else 2
+            v_count = 2
         self.B = {"q": Bar("q", 1), "ofinal": Bar("ofinal", 2), "list": Bar("list", 1)}
         for s in range(nk):
             self.B[f"kfull{s}"], self.B[f"kempty{s}"] = Bar(f"kfull{s}", 1), Bar(f"kempty{s}", 1)
         for s in range(nv):
-            self.B[f"vfull{s}"], self.B[f"vempty{s}"] = Bar(f"vfull{s}", 1), Bar(f"vempty{s}", 2)
+            self.B[f"vfull{s}"], self.B[f"vempty{s}"] = Bar(f"vfull{s}", 1), Bar(f"vempty{s}", v_count)
         for b in range(2):
             self.B[f"sfull{b}"] = Bar(f"sfull{b}", 1)
             self.B[f"pvdone{b}"] = Bar(f"pvdone{b}", pv_count)
@@ -56,14 +72,32 @@ class Protocol:
         self.V = [None] * nv
         self.O_busy = [0, 0]           # PVs in flight per accumulator
 
+    def buffer_of(self, g, t, bb):
+        """S buffer and its use index for global tile g = t-th tile of the unit. "split": buffer
+        g & 1, use g >> 1. "alternate": buffer t & 1 (the group), use bb[b] + (t >> 1), where bb
+        counts each buffer's uses in earlier units."""
+        if self.alt:
+            b = t & 1
+            return b, bb[b] + (t >> 1)
+        return g & 1, g >> 1
+
+    @staticmethod
+    def advance(bb, T):
+        bb[0] += (T + 1) >> 1
+        bb[1] += T >> 1
+
     # ---- event machinery
     def later(self, fn):
         self.seq += 1
         self.events.append((self.now + self.rng.choice([1, 2, 5, 20, 60]), self.seq, fn))
 
     def run(self):
-        roles = {"producer": self.producer(), "qk": self.qk_issuer(), "pv0": self.pv_issuer(0),
-                 "pv1": self.pv_issuer(1), "sm0": self.softmax(0), "sm1": self.softmax(1)}
+        if self.group_issuers:
+            roles = {"producer": self.producer(), "is0": self.group_issuer(0), "is1": self.group_issuer(1),
+                     "sm0": self.softmax(0), "sm1": self.softmax(1)}
+        else:
+            roles = {"producer": self.producer(), "qk": self.qk_issuer(), "pv0": self.pv_issuer(0),
+                     "pv1": self.pv_issuer(1), "sm0": self.softmax(0), "sm1": self.softmax(1)}
         waiting = dict.fromkeys(roles)
         done, at_sync = set(), set()
         while True:
@@ -134,15 +168,16 @@ class Protocol:
             base += T
 
     def qk_issuer(self):
-        base = 0
+        base, bb = 0, [0, 0]
         for u, T in enumerate(self.plan):
             yield ("wait", "list", u)
             yield ("wait", "q", u)
             for t in range(T):
                 g = base + t
-                b, s = g & 1, g % self.nk
+                s = g % self.nk
+                b, use = self.buffer_of(g, t, bb)
                 if t >= 2 and self.mut != "qk_skips_pvdone":
-                    yield ("wait", f"pvdone{b}", (g - 2) >> 1)
+                    yield ("wait", f"pvdone{b}", use - 1)
                 yield ("wait", f"kfull{s}", g // self.nk)
                 if self.S_busy[b]:
                     raise AssertionError(f"hazard: QK({g}) writes S{b} while {sorted(self.S_busy[b])} run")
@@ -160,15 +195,19 @@ class Protocol:
                 self.later(qk_done)
             yield ("sync",)
             base += T
+            self.advance(bb, T)
 
     def pv_issuer(self, grp):
-        base = 0
+        base, bb = 0, [0, 0]
         for u, T in enumerate(self.plan):
             yield ("wait", "list", u)
             for t in range(T):
                 g = base + t
-                b, s = g & 1, g % self.nv
-                yield ("wait", f"pfull{b}{grp}", g >> 1)
+                s = g % self.nv
+                b, use = self.buffer_of(g, t, bb)
+                if self.alt and b != grp:
+                    continue  # the other group's tile
+                yield ("wait", f"pfull{b}{grp}", use)
                 yield ("wait", f"vfull{s}", g // self.nv)
                 if self.S[b] is None or self.S[b][:2] != ("P", g):
                     raise AssertionError(f"hazard: PV{grp}({g}) finds {self.S[b]} in S{b}")
@@ -183,7 +222,7 @@ class Protocol:
                     if self.V[s] != g:
                         raise AssertionError(f"hazard: V stage {s} overwritten during PV({g})")
                     self.halves.setdefault((b, g), set()).add(grp)
-                    if self.halves[(b, g)] == {0, 1}:
+                    if self.halves[(b, g)] == ({grp} if self.alt else {0, 1}):
                         self.S[b] = ("P", g, True)
                     self.B[f"vempty{s}"].arrive()
                     self.B[f"pvdone{b}"].arrive()
@@ -197,9 +236,67 @@ class Protocol:
             self.later(final_commit)
             yield ("sync",)
             base += T
+            self.advance(bb, T)
+
+    def group_issuer(self, grp):
+        """One thread issues both products of group grp: for each of the group's tiles, QK^T into
+        S[grp], then (once P is written) PV into O_grp; the next QK^T waits for that PV."""
+        base, bb = 0, [0, 0]
+        for u, T in enumerate(self.plan):
+            yield ("wait", "list", u)
+            yield ("wait", "q", u)
+            for t in range(grp, T, 2):
+                g = base + t
+                b, use = self.buffer_of(g, t, bb)
+                sk, sv = g % self.nk, g % self.nv
+                if t >= 2 and self.mut != "qk_skips_pvdone":
+                    yield ("wait", f"pvdone{b}", use - 1)
+                yield ("wait", f"kfull{sk}", g // self.nk)
+                if self.S_busy[b]:
+                    raise AssertionError(f"hazard: QK({g}) writes S{b} while {sorted(self.S_busy[b])} run")
+                if self.S[b] is not None and self.S[b][0] == "P" and not self.S[b][2]:
+                    raise AssertionError(f"hazard: QK({g}) overwrites P({self.S[b][1]}) before its PV completed")
+                if self.K[sk] != g:
+                    raise AssertionError(f"hazard: QK({g}) reads K stage {sk} holding tile {self.K[sk]}")
+                self.S_busy[b].add(("QK", g))
+
+                def qk_done(b=b, s=sk, g=g):
+                    self.S_busy[b].discard(("QK", g))
+                    self.S[b] = ("S", g, False)
+                    self.B[f"sfull{b}"].arrive()
+                    self.B[f"kempty{s}"].arrive()
+                self.later(qk_done)
+                yield ("wait", f"pfull{b}{grp}", use)
+                yield ("wait", f"vfull{sv}", g // self.nv)
+                if self.S[b] is None or self.S[b][:2] != ("P", g):
+                    raise AssertionError(f"hazard: PV{grp}({g}) finds {self.S[b]} in S{b}")
+                if self.V[sv] != g:
+                    raise AssertionError(f"hazard: PV{grp}({g}) reads V stage {sv} holding tile {self.V[sv]}")
+                self.S_busy[b].add(("PV", g, grp))
+                self.O_busy[grp] += 1
+
+                def pv_done(b=b, s=sv, g=g):
+                    self.S_busy[b].discard(("PV", g, grp))
+                    self.O_busy[grp] -= 1
+                    if self.V[s] != g:
+                        raise AssertionError(f"hazard: V stage {s} overwritten during PV({g})")
+                    self.S[b] = ("P", g, True)
+                    self.B[f"vempty{s}"].arrive()
+                    self.B[f"pvdone{b}"].arrive()
+                self.later(pv_done)
+
+            def final_commit():
+                if self.O_busy[grp]:
+                    self.later(final_commit)
+                else:
+                    self.B["ofinal"].arrive()
+            self.later(final_commit)
+            yield ("sync",)
+            base += T
+            self.advance(bb, T)
 
     def softmax(self, grp):
-        base = 0
+        base, bb = 0, [0, 0]
         for u, T in enumerate(self.plan):
             if self.route_in_kernel:
                 yield ("wait", "q", u)  # q_bar comes from the Q tile in shared memory
@@ -207,12 +304,23 @@ class Protocol:
                 self.B["list"].arrive()  # thread 0 of the softmax warps publishes the tile lists
             else:
                 yield ("wait", "list", u)
+            started = False
             for t in range(T):
                 g = base + t
-                b = g & 1
-                yield ("wait", f"sfull{b}", g >> 1)
+                b, use = self.buffer_of(g, t, bb)
+                if self.alt and b != grp:
+                    continue  # the other group's tile
+                yield ("wait", f"sfull{b}", use)
                 if self.S[b] is None or self.S[b][:2] not in (("S", g), ("P", g)):
                     raise AssertionError(f"hazard: softmax{grp}({g}) finds {self.S[b]} in S{b}")
+                if self.alt:
+                    # a lazy rescale may come at any tile after the group's first: O_grp must be at rest
+                    if started and self.rng.random() < 0.5 and self.O_busy[grp]:
+                        raise AssertionError(f"hazard: rescale of O{grp} at tile {g} with a PV in flight")
+                    started = True
+                    self.S[b] = ("P", g, False)
+                    self.B[f"pfull{b}{grp}"].arrive()
+                    continue
                 if t > 0 and self.rng.random() < 0.3:
                     # a lazy rescale of O_grp: wait for the previous tile's PVs, then O_grp must be at rest
                     yield ("wait", f"pvdone{(g - 1) & 1}", (g - 1) >> 1)
@@ -226,6 +334,7 @@ class Protocol:
                     raise AssertionError("hazard: the epilogue reads O with a PV in flight")
             yield ("sync",)
             base += T
+            self.advance(bb, T)
 
 
 def random_plan(rng):

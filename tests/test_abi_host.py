@@ -97,6 +97,9 @@ def test_pool_rejects_invalid_arguments(lib):
     assert lib.sol_attn_pool(p[0], p[1], sa.SOL_BF16, 1, 1, 100, 64, 128, p[2], p[3], None, None, None) == sa.SOL_EINVAL
     assert lib.sol_attn_pool(p[0], p[1], sa.SOL_F32, 1, 1, 100, 64, 128, p[2], p[3], p[4], p[5], None) == sa.SOL_EINVAL
     assert lib.sol_attn_pool(p[0], p[1], sa.SOL_BF16, 1, 1, 100, 60, 128, p[2], p[3], p[4], p[5], None) == sa.SOL_EUNSUPPORTED
+    # rows of 12 or 64 16-byte vectors: not a power of two <= 32
+    assert lib.sol_attn_pool(p[0], p[1], sa.SOL_BF16, 1, 1, 100, 96, 128, p[2], p[3], p[4], p[5], None) == sa.SOL_EUNSUPPORTED
+    assert lib.sol_attn_pool(p[0], p[1], sa.SOL_F32, 1, 1, 100, 256, 128, p[2], p[3], None, None, None) == sa.SOL_EUNSUPPORTED
     assert lib.sol_attn_pool(p[0], p[1], sa.SOL_BF16, 1, 1, 0, 64, 128, p[2], p[3], p[4], p[5], None) == sa.SOL_EINVAL
 
 

@@ -67,7 +67,8 @@ def check_mask_density(mask, dens, n_force=0):
 # ------------------------------------------------------------------------------------------------
 
 @pytest.mark.parametrize("dtype,L,d,blk", [("bf16", 1000, 128, 128), ("bf16", 77, 64, 128), ("f32", 1000, 64, 64),
-                                           ("bf16", 4096, 128, 128), ("f32", 130, 128, 32)])
+                                           ("bf16", 4096, 128, 128), ("f32", 130, 128, 32), ("bf16", 300, 256, 128),
+                                           ("bf16", 260, 8, 64), ("f32", 99, 4, 16), ("f32", 500, 32, 128)])
 def test_pool_matches_oracle(dtype, L, d, blk):
     rng = np.random.default_rng(L + d)
     B, H = 2, 3

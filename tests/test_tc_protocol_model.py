@@ -1,10 +1,11 @@
 """The fused kernel's mbarrier protocol, run as a discrete-event model (tests/tc_protocol_model.py).
 
 Random unit sizes (including one-tile units) and random completion delays, for the ring depths
-of both head dimensions: no deadlock, no stale parity wait, no data hazard. Three planted protocol
-mistakes must each be caught: a QK^T that does not wait for the PVs two tiles back, a PV-done
-barrier completed by one group instead of both, and a producer that waits for the V stage's
-use before the previous one.
+of both head dimensions and both schedules (groups on alternate tiles, the kernel's; groups on
+column halves of every tile): no deadlock, no stale parity wait, no data hazard. Planted protocol
+mistakes must each be caught: a QK^T that does not wait for the PV two tiles back, a PV-done
+barrier with the wrong arrival count, and a producer that waits for the V stage's use before the
+previous one.
 """
 import random
 
@@ -13,21 +14,27 @@ import pytest
 from tc_protocol_model import Protocol, random_plan
 
 
+@pytest.mark.parametrize("schedule", ["group_issuers", "alternate", "split"])
 @pytest.mark.parametrize("nk,nv", [(3, 2), (4, 4)])  # d = 128 and d = 64 ring depths
 @pytest.mark.parametrize("route_in_kernel", [False, True])  # keep bits from the routing pass, or routed in place
-def test_protocol_has_no_deadlock_stale_wait_or_hazard(nk, nv, route_in_kernel):
+def test_protocol_has_no_deadlock_stale_wait_or_hazard(nk, nv, route_in_kernel, schedule):
     rng = random.Random(nk * 10 + nv)
     for k in range(150):
-        Protocol(random_plan(rng), seed=k, nk=nk, nv=nv, route_in_kernel=route_in_kernel).run()
+        Protocol(random_plan(rng), seed=k, nk=nk, nv=nv, route_in_kernel=route_in_kernel, schedule=schedule).run()
 
 
-@pytest.mark.parametrize("mutation", ["qk_skips_pvdone", "pvdone_count_1", "vempty_one_back"])
-def test_planted_protocol_mistakes_are_caught(mutation):
+@pytest.mark.parametrize("schedule,mutation", [
+    ("split", "qk_skips_pvdone"), ("split", "pvdone_count_1"), ("split", "vempty_one_back"),
+    ("alternate", "qk_skips_pvdone"), ("alternate", "alt_pvdone_count_2"), ("alternate", "vempty_one_back"),
+    ("group_issuers", "qk_skips_pvdone"), ("group_issuers", "alt_pvdone_count_2"),
+    ("group_issuers", "vempty_one_back"),
+])
+def test_planted_protocol_mistakes_are_caught(schedule, mutation):
     rng = random.Random(5)
     caught = 0
     for k in range(150):
         try:
-            Protocol(random_plan(rng), seed=k, mutation=mutation).run()
+            Protocol(random_plan(rng), seed=k, mutation=mutation, schedule=schedule).run()
         except AssertionError:
             caught += 1
     assert caught > 0
