@@ -363,6 +363,51 @@ def cta_spans(launch, dev, torch, sa):
             "tail_frac": float((end.max() - end.mean()) / span), "busy_frac": float(((end - start) / span).mean())}
 
 
+def measure_int8_qk(w, Q, K, V, kbar, vlp, tau, O_bf16, ws, stream, flops, bf16_fwd_ms, pk, max_over_ranks, barrier,
+                    world):
+    """The 8-bit QK^T variant on the workload at the timed density: CUDA-event time of the
+    quantization pass and of the forward, kept-tile TFLOP/s of the forward (the same FLOP count
+    as the bf16 line), its ratio to the bf16 forward, and its output's distance from the bf16
+    output (the variant's own quantization error)."""
+    import torch
+    from block_sparse_attention_41_b200 import sol_attn as sa
+    q8, k8, kb8, qs, ks, kbs, mu = sa.sol_attn_quantize_qk8(Q, K, kbar, stream=stream)
+    O8 = torch.empty_like(Q)
+
+    def quant():
+        sa.sol_attn_quantize_qk8(Q, K, kbar, stream=stream)
+
+    def fwd():
+        sa.sol_attn_fwd_qk8(Q, q8, k8, kb8, qs, ks, kbs, V, kbar, vlp, tau, w.n_force, O=O8, workspace=ws,
+                            stream=stream)
+
+    def timed(fn, n_it=5):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        barrier()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_it)]
+        for a, b in ev:
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ev))
+
+    q_ms = timed(quant)
+    f_ms = timed(fwd)
+    sa.sol_attn_check_device_error(ws)
+    diff = (O8.float() - O_bf16.float()).abs()
+    tflops = flops / (f_ms * 1e-3) / 1e12
+    out = {"kernel": "sol_fwd_tc_kernel<128, int8 QK^T>", "quantize_ms": q_ms, "fwd_ms": f_ms,
+           "fwd_tflops": world * tflops, "frac_of_bf16_peak": tflops / pk["bf16_tflops"],
+           "speedup_vs_bf16_fwd": bf16_fwd_ms / f_ms,
+           "vs_bf16_output": {"max_abs": float(diff.max()), "mean_abs": float(diff.mean())},
+           "note": "QK^T on int8 tensor cores (kind::i8), PV in bf16; FLOPs counted as for the bf16 line"}
+    del q8, k8, kb8, O8, diff
+    return out
+
+
 def per_run_report(w, Q, K, V, kbar, vbar, klp, vlp, tau, key, O, dens, ws, stream):
     """One untimed call with the kept mask: per-head densities, kept-tile FLOPs over valid tokens
     only (the partial last query and key blocks count their valid rows and columns), the
@@ -584,6 +629,11 @@ def run_ours(args, w):
         next_rows = {"qknorm_rope_pool": measure_qknorm_rope_pool(
             w, Q, K, V, stream, pk, rank == 0 and world == 1 and not args.no_cpu_baseline, max_over_ranks, barrier,
             world)}
+        if w.d == 128:
+            step(tau)  # the sweep left another density's output in O
+            torch.cuda.synchronize()
+            next_rows["int8_qk"] = measure_int8_qk(w, Q, K, V, kbar, vlp, tau, O, ws, stream, flops, fwd_ms, pk,
+                                                   max_over_ranks, barrier, world)
 
     # end to end through the public API: pinned host inputs in, host output back, every step. The
     # host-buffer entry point uploads, computes and downloads chunks of heads concurrently.
@@ -666,7 +716,7 @@ def run_ours(args, w):
                      "frac": pool_bytes / (pool_ms * 1e-3) / 1e9 / pk["hbm_gbs"]},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": 3 * args.steps,  # pool, routing pass, fused forward
+            "gpu_launches": 4 * args.steps,  # pool, q_bar, routing kernel, fused forward
             "clocks": clocks,
             "sweep": sweep,
             "next_rows": next_rows,

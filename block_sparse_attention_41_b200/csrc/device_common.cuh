@@ -177,6 +177,17 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::i8 (signed 8-bit inputs, 32-bit integer accumulate).
+__device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand (sm_100 format: version 1).
 // lbo/sbo are byte offsets: K-major uses sbo = 1024 (8 rows of 128 B) and ignores lbo; MN-major
 // uses lbo = distance between 64-element MN groups and sbo = distance between 8-row K groups.
@@ -198,6 +209,21 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
          | ((b_mn_major ? 1u : 0u) << 16)            // B major-ness
          | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+// Instruction descriptor, kind::i8 with signed 8-bit A/B and signed 32-bit D; A and B K-major.
+__host__ __device__ constexpr uint32_t idesc_s8_s32(int M, int N) {
+  return (2u << 4)                                   // D format: s32
+         | (1u << 7)                                 // A format: signed 8-bit
+         | (1u << 10)                                // B format: signed 8-bit
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+// An int32 accumulator value as fp32, exactly for |i| < 2^22: the integer is added to the bit
+// pattern of 1.5 * 2^23, whose float spacing is 1, and 1.5 * 2^23 is subtracted back.
+__device__ __forceinline__ float s32_to_f32_small(uint32_t raw) {
+  return __int_as_float(static_cast<int>(raw) + 0x4B400000) - 12582912.0f;
 }
 
 // Per-warpgroup register re-balancing (all warps of a warpgroup execute the same one).

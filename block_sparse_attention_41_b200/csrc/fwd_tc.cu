@@ -76,16 +76,20 @@ constexpr float kExpC1 = 0.69511664f, kExpC2 = 0.22764498f, kExpC3 = 0.07706724f
 // MUFU costs more issue slots than it saves, so it is off.
 constexpr int kPolyEvery = 0;
 
-template <int D>
+// QK8: Q, K and the pooled keys arrive as int8 codes (one 128-byte swizzle atom per row at d = 128)
+// and QK^T runs as kind::i8 with int32 accumulation; V, P and the rest stay bf16.
+template <int D, bool QK8>
 struct TcCfg {
-  static constexpr int NCHUNK = D / 64;                 // 128-byte swizzle atoms per row
+  static constexpr int NCHUNK = D / 64;                 // 128-byte swizzle atoms per bf16 row
   static constexpr int CHUNK_BYTES = kRows * 128;       // 128 rows x 128 B
   static constexpr int TILE_BYTES = NCHUNK * CHUNK_BYTES;
+  static constexpr int QK_CHUNKS = QK8 ? D / 128 : NCHUNK;  // swizzle atoms per Q or K row
+  static constexpr int QK_TILE_BYTES = QK_CHUNKS * CHUNK_BYTES;
   static constexpr int NK = (D == 128) ? 3 : 4;         // K ring depth
   static constexpr int NV = (D == 128) ? 2 : 4;         // V ring depth
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + TILE_BYTES;
-  static constexpr int OFF_V = OFF_K + NK * TILE_BYTES;
+  static constexpr int OFF_K = OFF_Q + QK_TILE_BYTES;
+  static constexpr int OFF_V = OFF_K + NK * QK_TILE_BYTES;
   static constexpr int OFF_SBAR = OFF_V + NV * TILE_BYTES;                // float[kMaxKeyBlocks]
   static constexpr int OFF_KLIST = OFF_SBAR + kMaxKeyBlocks * 4;          // u16[kMaxKeyBlocks]
   static constexpr int OFF_BITS = OFF_KLIST + kMaxKeyBlocks * 2;          // u32[kMaxKeyBlocks/32]
@@ -104,6 +108,7 @@ struct TcCfg {
   static_assert(kMaxKeyBlocks / 32 <= kSoftmaxThreads, "word prefixes fit after q_bar");
   static_assert((kSoftmaxThreads / (D / 8)) * D <= kMaxKeyBlocks, "q_bar partial sums fit in the proxy-score buffer");
   static_assert(kColO + 2 * D <= kTmemCols, "TMEM budget");
+  static_assert(!QK8 || D == 128, "8-bit QK^T needs d = 128");
 };
 
 struct TcParams {
@@ -119,6 +124,9 @@ struct TcParams {
   float log2_last_n;
   int drop_one_load;
   unsigned long long wait_limit_ns;
+  const float* q_scale;   // 8-bit QK^T: [BH, nqb] query-tile scales
+  const float* k_scale;   // [BH, nkb] key-block scales
+  const float* kb_scale;  // [BH, ceil(nkb / 128)] pooled-key chunk scales
   unsigned long long* cta_times;  // measurement hook: [2 * cta_capacity] start/finish ns, or null
   int cta_capacity;
   float tau[kMaxHeads];
@@ -152,12 +160,12 @@ __device__ __forceinline__ float max64(const float (&s)[64]) {
   return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
 
-template <int D>
+template <int D, bool QK8>
 __global__ void __launch_bounds__(kThreads, 1)
     sol_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKb,
                       const __grid_constant__ CUtensorMap tmVb, const __grid_constant__ TcParams p) {
-  using C = TcCfg<D>;
+  using C = TcCfg<D, QK8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -245,9 +253,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
       // ------------------------------------------------------------------ TMA producer
       if (lane == 0) {
-        mbar_arrive_expect_tx(bar_q, C::TILE_BYTES);
-        for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_3d(sb + C::OFF_Q + c * C::CHUNK_BYTES, &tmQ, bar_q, c * 64, qb * kRows, bh);
+        mbar_arrive_expect_tx(bar_q, C::QK_TILE_BYTES);
+        for (int c = 0; c < C::QK_CHUNKS; ++c)  // a 128-byte-wide box: 64 bf16 or 128 int8 columns
+          tma_load_3d(sb + C::OFF_Q + c * C::CHUNK_BYTES, &tmQ, bar_q, c * (QK8 ? 128 : 64), qb * kRows, bh);
         int w = mbar_wait(bar_list, uphase, s_abort, limit);
         if (w == WAIT_TIMEOUT) raise_timeout(s_abort, p.ws, WHERE_PRODUCER);
         if (w == WAIT_OK) {
@@ -269,10 +277,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int y = (exact ? static_cast<int>(s_klist[t]) : static_cast<int>(s_clist[t - nk])) * kRows;
               const bool drop = p.drop_one_load && blockIdx.x == 0 && unit_iter == 0 && t == 0;
               if (!drop) {
-                mbar_arrive_expect_tx(bar_kfull + 8 * s, C::TILE_BYTES);
-                for (int c = 0; c < C::NCHUNK; ++c)
-                  tma_load_3d(sb + C::OFF_K + s * C::TILE_BYTES + c * C::CHUNK_BYTES, mk, bar_kfull + 8 * s, c * 64,
-                              y, bh);
+                mbar_arrive_expect_tx(bar_kfull + 8 * s, C::QK_TILE_BYTES);
+                for (int c = 0; c < C::QK_CHUNKS; ++c)
+                  tma_load_3d(sb + C::OFF_K + s * C::QK_TILE_BYTES + c * C::CHUNK_BYTES, mk, bar_kfull + 8 * s,
+                              c * (QK8 ? 128 : 64), y, bh);
                 k_armed[s] = g / C::NK + 1u;
               }
             }
@@ -340,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (w == WAIT_OK) w = mbar_wait(bar_q, uphase, s_abort, limit);
         if (w == WAIT_OK) {
           const int T = s_misc[MISC_NK] + s_misc[MISC_NC];
-          constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
+          constexpr uint32_t idesc_qk = QK8 ? idesc_s8_s32(128, 128) : idesc_bf16_f32(128, 128, false);
           const uint64_t qdesc0 = smem_desc_sw128(sb + C::OFF_Q, 16, 1024);
           const uint64_t kdesc0 = smem_desc_sw128(sb + C::OFF_K, 16, 1024);
           for (int t = 0; t < T && w == WAIT_OK; ++t) {
@@ -354,11 +362,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (w == WAIT_OK) w = mbar_wait(bar_kfull + 8 * s, (g / C::NK) & 1u, s_abort, limit);
             if (w != WAIT_OK) break;
             tc_fence_after();
-            const uint64_t kd = kdesc0 + ((s * C::TILE_BYTES) >> 4);
+            const uint64_t kd = kdesc0 + ((s * C::QK_TILE_BYTES) >> 4);
+            if constexpr (QK8) {
+              // K = 32 int8 values (32 bytes) per MMA: four steps through the row's single atom
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = ((kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32) >> 4;
-              mma_bf16_ss(tmem + kColS + 128 * b, qdesc0 + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < D / 32; ++kk)
+                mma_i8_ss(tmem + kColS + 128 * b, qdesc0 + kk * 2, kd + kk * 2, idesc_qk, kk > 0 ? 1u : 0u);
+            } else {
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = ((kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32) >> 4;
+                mma_bf16_ss(tmem + kColS + 128 * b, qdesc0 + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
+              }
             }
             mma_issued = true;
             tc_commit(bar_sfull + 8 * b);
@@ -537,6 +552,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
+      if constexpr (QK8) {
+        // the scale of each kept tile's int32 scores: log2(e)/sqrt(d) * scale_q * scale_k. The
+        // proxy-score buffer is free: 8-bit QK^T always comes with the routing pass's bits.
+        const float sq = p.sl2 * __ldg(p.q_scale + unit);
+        const float* ks = p.k_scale + static_cast<size_t>(bh) * nkb;
+        const int nk_u = s_misc[MISC_NK];
+        for (int t = st; t < nk_u; t += kSoftmaxThreads) s_sbar[t] = sq * __ldg(ks + s_klist[t]);
+        named_barrier_sync(kBarSoftmax, kSoftmaxThreads);
+      }
       if (st == 0 && alive) mbar_arrive(bar_list);
       if (p.kept_mask != nullptr && p.bits == nullptr) {
         uint8_t* mrow = p.kept_mask + (static_cast<size_t>(bh) * p.nqb + qb) * nkb;
@@ -549,6 +573,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nk = s_misc[MISC_NK];
       const int T = alive ? nk + s_misc[MISC_NC] : 0;
       const float sl2 = p.sl2;
+      // 8-bit QK^T: pooled tiles take log2(e)/sqrt(d) * scale_q * scale of their chunk of pooled keys
+      const float sq2 = QK8 ? sl2 * __ldg(p.q_scale + unit) : sl2;
+      const float* kbs = QK8 ? p.kb_scale + static_cast<size_t>(bh) * ((nkb + kRows - 1) / kRows) : nullptr;
       const uint32_t o_col = tmem + lane_base + kColO + D * grp;
       float m_run = -INFINITY, l_run = 0.f;
       bool bad = false;  // a wait of this warp failed inside the tile loop
@@ -567,20 +594,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool exact = t < nk;
         const int j = exact ? static_cast<int>(s_klist[t]) : 0;
         const bool full = exact && (j != nkb - 1 || p.last_n == kRows);
+        // the factor that turns this tile's raw scores into log2-domain logits (> 0)
+        float ts = sl2;
+        if constexpr (QK8) ts = exact ? s_sbar[t] : sq2 * __ldg(kbs + s_clist[t - nk]);
         {
           uint32_t raw[64];
           tmem_ld_x64(s_col, raw);
 #pragma unroll
-          for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(raw[c]);
+          for (int c = 0; c < 64; ++c) s[c] = QK8 ? s32_to_f32_small(raw[c]) : __uint_as_float(raw[c]);
         }
         float mx;
         if (full) {
-          mx = max64(s) * sl2;  // sl2 > 0: the max of the scaled scores
+          mx = max64(s) * ts;  // ts > 0: the max of the scaled scores
         } else {
           if (exact) {
             const int valid = p.last_n - grp * 64;  // valid columns in this half (may be <= 0)
 #pragma unroll
-            for (int c = 0; c < 64; ++c) s[c] = (c < valid) ? s[c] * sl2 : -INFINITY;
+            for (int c = 0; c < 64; ++c) s[c] = (c < valid) ? s[c] * ts : -INFINITY;
           } else {
             const int cc = s_clist[t - nk];
             const int valid = min(kRows, nkb - cc * kRows) - grp * 64;
@@ -593,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t kw = c < 32 ? kw0 : kw1;
               const bool skipped = c < valid && !((kw >> (c & 31)) & 1u);
               const float off = (c == last_col) ? p.log2_last_n : 7.0f;  // log2(n_j)
-              s[c] = skipped ? fmaf(s[c], sl2, off) : -INFINITY;
+              s[c] = skipped ? fmaf(s[c], ts, off) : -INFINITY;
             }
           }
           mx = max64(s);
@@ -614,7 +644,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pk[32];
         float acc[4] = {0.f, 0.f, 0.f, 0.f};  // row sum of the bf16-rounded weights, 4 chains
         if (full) {
-          const float2 scale2 = make_float2(sl2, sl2);
+          const float2 scale2 = make_float2(ts, ts);
           const float2 negm2 = make_float2(-m_use, -m_use);
 #pragma unroll
           for (int c2 = 0; c2 < 32; ++c2) {
@@ -753,9 +783,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
+template <int D, bool QK8>
 cudaError_t launch_tc_t(const FwdArgs& a, const CUtensorMap* maps, cudaStream_t stream) {
-  using C = TcCfg<D>;
+  using C = TcCfg<D, QK8>;
   TcParams p;
   p.kbar = a.kbar;
   p.bits = a.route_bits;
@@ -776,23 +806,31 @@ cudaError_t launch_tc_t(const FwdArgs& a, const CUtensorMap* maps, cudaStream_t 
   p.log2_last_n = static_cast<float>(std::log2(static_cast<double>(p.last_n)));
   p.drop_one_load = a.drop_one_load;
   p.wait_limit_ns = a.wait_limit_ns;
+  p.q_scale = QK8 ? a.qk8->q_scale : nullptr;
+  p.k_scale = QK8 ? a.qk8->k_scale : nullptr;
+  p.kb_scale = QK8 ? a.qk8->kb_scale : nullptr;
   p.cta_times = a.cta_times;
   p.cta_capacity = a.cta_capacity;
   for (int h = 0; h < kMaxHeads; ++h) p.tau[h] = h < a.H ? a.tau[h] : 0.f;
-  cudaError_t e = cudaFuncSetAttribute(sol_fwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(sol_fwd_tc_kernel<D, QK8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int grid = p.total_units < a.num_sms ? p.total_units : a.num_sms;
-  sol_fwd_tc_kernel<D><<<grid, kThreads, C::SMEM_BYTES, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
+  sol_fwd_tc_kernel<D, QK8><<<grid, kThreads, C::SMEM_BYTES, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_fwd_tc(const FwdArgs& a, const CUtensorMap* maps, cudaStream_t stream) {
-  if (a.qk8 != nullptr) return cudaErrorNotSupported;
-  if (a.d == 64) return launch_tc_t<64>(a, maps, stream);
-  if (a.d == 128) return launch_tc_t<128>(a, maps, stream);
+  if (a.qk8 != nullptr) {
+    // 8-bit QK^T: d = 128 and keep bits from the routing pass (the Q tile in shared memory holds
+    // int8 codes, which the in-kernel routing cannot average)
+    if (a.d != 128 || a.route_bits == nullptr) return cudaErrorNotSupported;
+    return launch_tc_t<128, true>(a, maps, stream);
+  }
+  if (a.d == 64) return launch_tc_t<64, false>(a, maps, stream);
+  if (a.d == 128) return launch_tc_t<128, false>(a, maps, stream);
   return cudaErrorInvalidValue;
 }
 

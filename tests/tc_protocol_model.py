@@ -45,8 +45,10 @@ class Protocol:
     def __init__(self, plan, seed, nk=3, nv=2, mutation=None, route_in_kernel=False, schedule="split"):
         self.plan, self.nk, self.nv, self.mut = plan, nk, nv, mutation
         self.route_in_kernel = route_in_kernel  # no keep bits given: the softmax warps route from the Q tile
-        self.alt = schedule in ("alternate", "group_issuers")
+        self.alt = schedule in ("alternate", "group_issuers", "smem_p")
         self.group_issuers = schedule == "group_issuers"
+        self.smem_p = schedule == "smem_p"
+        self.dephase = schedule == "split_dephase"
         self.rng = random.Random(seed)
         self.now, self.seq, self.events = 0, 0, []
         if self.alt:  # one PV per tile: the owning group's
@@ -62,6 +64,8 @@ class Protocol:
             self.B[f"vfull{s}"], self.B[f"vempty{s}"] = Bar(f"vfull{s}", 1), Bar(f"vempty{s}", v_count)
         for b in range(2):
             self.B[f"sfull{b}"] = Bar(f"sfull{b}", 1)
+            self.B[f"sfree{b}"] = Bar(f"sfree{b}", 2 if schedule == "split_dephase" else 1)
+            self.B[f"pvg{b}"] = Bar(f"pvg{b}", 1)
             self.B[f"pvdone{b}"] = Bar(f"pvdone{b}", pv_count)
             for grp in range(2):
                 self.B[f"pfull{b}{grp}"] = Bar(f"pfull{b}{grp}", 1)
@@ -71,6 +75,9 @@ class Protocol:
         self.K = [None] * nk
         self.V = [None] * nv
         self.O_busy = [0, 0]           # PVs in flight per accumulator
+        self.P = [None, None]          # smem_p: tile whose P a group's shared-memory buffer holds
+        self.P_busy = [0, 0]           # smem_p: PVs in flight reading each P buffer
+        self.S_read = [None, None]     # smem_p: last tile whose S the group has read out of TMEM
 
     def buffer_of(self, g, t, bb):
         """S buffer and its use index for global tile g = t-th tile of the unit. "split": buffer
@@ -92,7 +99,13 @@ class Protocol:
         self.events.append((self.now + self.rng.choice([1, 2, 5, 20, 60]), self.seq, fn))
 
     def run(self):
-        if self.group_issuers:
+        if self.dephase:
+            roles = {"producer": self.producer(), "qk": self.dephase_qk(), "pv0": self.dephase_pv(0),
+                     "pv1": self.dephase_pv(1), "sm0": self.dephase_softmax(0), "sm1": self.dephase_softmax(1)}
+        elif self.smem_p:
+            roles = {"producer": self.producer(), "is0": self.smem_issuer(0), "is1": self.smem_issuer(1),
+                     "sm0": self.smem_softmax(0), "sm1": self.smem_softmax(1)}
+        elif self.group_issuers:
             roles = {"producer": self.producer(), "is0": self.group_issuer(0), "is1": self.group_issuer(1),
                      "sm0": self.softmax(0), "sm1": self.softmax(1)}
         else:
@@ -291,6 +304,218 @@ class Protocol:
                 else:
                     self.B["ofinal"].arrive()
             self.later(final_commit)
+            yield ("sync",)
+            base += T
+            self.advance(bb, T)
+
+    # ---- split columns, P in shared memory, group 1 a phase behind
+    def dephase_qk(self):
+        base = 0
+        self.reads = {}  # tile -> groups that have read their half of its S
+        for u, T in enumerate(self.plan):
+            yield ("wait", "list", u)
+            yield ("wait", "q", u)
+            for t in range(T):
+                g = base + t
+                b, s = g & 1, g % self.nk
+                if t >= 2 and self.mut != "qk_skips_sfree":
+                    yield ("wait", f"sfree{b}", (g - 2) >> 1)
+                yield ("wait", f"kfull{s}", g // self.nk)
+                if self.S_busy[b]:
+                    raise AssertionError(f"hazard: QK({g}) writes S{b} while {sorted(self.S_busy[b])} run")
+                if self.S[b] is not None and self.reads.get(self.S[b][1], set()) != {0, 1}:
+                    raise AssertionError(f"hazard: QK({g}) overwrites S({self.S[b][1]}) before both halves were read")
+                if self.K[s] != g:
+                    raise AssertionError(f"hazard: QK({g}) reads K stage {s} holding tile {self.K[s]}")
+                self.S_busy[b].add(("QK", g))
+
+                def qk_done(b=b, s=s, g=g):
+                    self.S_busy[b].discard(("QK", g))
+                    self.S[b] = ("S", g, False)
+                    self.B[f"sfull{b}"].arrive()
+                    self.B[f"kempty{s}"].arrive()
+                self.later(qk_done)
+            yield ("sync",)
+            base += T
+
+    def dephase_pv(self, grp):
+        base = 0
+        for u, T in enumerate(self.plan):
+            yield ("wait", "list", u)
+            for t in range(T):
+                g = base + t
+                b, s = g & 1, g % self.nv
+                yield ("wait", f"pfull{b}{grp}", g >> 1)
+                yield ("wait", f"vfull{s}", g // self.nv)
+                if self.P[grp] != g:
+                    raise AssertionError(f"hazard: PV{grp}({g}) finds P of {self.P[grp]}")
+                if self.V[s] != g:
+                    raise AssertionError(f"hazard: PV{grp}({g}) reads V stage {s} holding tile {self.V[s]}")
+                self.P_busy[grp] += 1
+                self.O_busy[grp] += 1
+
+                def pv_done(s=s, g=g):
+                    self.P_busy[grp] -= 1
+                    self.O_busy[grp] -= 1
+                    if self.V[s] != g:
+                        raise AssertionError(f"hazard: V stage {s} overwritten during PV({g})")
+                    self.B[f"vempty{s}"].arrive()
+                    self.B[f"pvg{grp}"].arrive()
+                self.later(pv_done)
+
+            def final_commit():
+                if self.O_busy[grp]:
+                    self.later(final_commit)
+                else:
+                    self.B["ofinal"].arrive()
+            self.later(final_commit)
+            yield ("sync",)
+            base += T
+
+    def dephase_softmax(self, grp):
+        base = 0
+        for u, T in enumerate(self.plan):
+            if self.route_in_kernel:
+                yield ("wait", "q", u)
+            if grp == 0:
+                self.B["list"].arrive()
+            else:
+                yield ("wait", "list", u)
+
+            def read(g, release):
+                b = g & 1
+                if self.S[b] is None or self.S[b][:2] != ("S", g):
+                    raise AssertionError(f"hazard: softmax{grp}({g}) finds {self.S[b]} in S{b}")
+                if release:
+                    self.reads.setdefault(g, set()).add(grp)
+                    self.B[f"sfree{b}"].arrive()
+
+            def weights(t):
+                g = base + t
+                if grp == 1:
+                    read(g, True)  # the scores are read again, then released
+                if t >= 1 and self.mut != "p_skips_pvdone":
+                    yield ("wait", f"pvg{grp}", g - 1)
+                if self.P_busy[grp]:
+                    raise AssertionError(f"hazard: softmax{grp}({g}) overwrites P while a PV reads it")
+                if self.O_busy[grp]:
+                    raise AssertionError(f"hazard: rescale of O{grp} at tile {g} with a PV in flight")
+                self.P[grp] = g
+                self.B[f"pfull{g & 1}{grp}"].arrive()
+
+            def maxes(t):
+                g = base + t
+                yield ("wait", f"sfull{g & 1}", g >> 1)
+                read(g, grp == 0)
+
+            for it in range(T + grp):
+                if grp == 1 and it >= 1:
+                    yield from weights(it - 1)
+                if it < T:
+                    yield from maxes(it)
+                if grp == 0:
+                    yield from weights(it)
+            if T > 0:
+                yield ("wait", "ofinal", u)
+                if any(self.O_busy):
+                    raise AssertionError("hazard: the epilogue reads O with a PV in flight")
+            yield ("sync",)
+            base += T
+
+    def smem_issuer(self, grp):
+        """Group grp's issuer with P in shared memory: the next QK^T into S[grp] waits only for the
+        softmax to have read S out of TMEM; the PV reads P from the group's shared buffer."""
+        base, bb = 0, [0, 0]
+        for u, T in enumerate(self.plan):
+            yield ("wait", "list", u)
+            yield ("wait", "q", u)
+
+            def qk(t):
+                g = base + t
+                sk = g % self.nk
+                yield ("wait", f"kfull{sk}", g // self.nk)
+                if self.S_busy[grp]:
+                    raise AssertionError(f"hazard: QK({g}) writes S{grp} while {sorted(self.S_busy[grp])} run")
+                if self.S[grp] is not None and self.S[grp][0] == "S" and self.S_read[grp] != self.S[grp][1]:
+                    raise AssertionError(f"hazard: QK({g}) overwrites S({self.S[grp][1]}) before it was read")
+                if self.K[sk] != g:
+                    raise AssertionError(f"hazard: QK({g}) reads K stage {sk} holding tile {self.K[sk]}")
+                self.S_busy[grp].add(("QK", g))
+
+                def qk_done(s=sk, g=g):
+                    self.S_busy[grp].discard(("QK", g))
+                    self.S[grp] = ("S", g, False)
+                    self.B[f"sfull{grp}"].arrive()
+                    self.B[f"kempty{s}"].arrive()
+                self.later(qk_done)
+            if grp < T:
+                yield from qk(grp)
+            for t in range(grp, T, 2):
+                g = base + t
+                _, use = self.buffer_of(g, t, bb)
+                if t + 2 < T:
+                    if self.mut != "qk_skips_sfree":
+                        yield ("wait", f"sfree{grp}", use)
+                    yield from qk(t + 2)
+                sv = g % self.nv
+                yield ("wait", f"pfull{grp}{grp}", use)
+                yield ("wait", f"vfull{sv}", g // self.nv)
+                if self.P[grp] != g:
+                    raise AssertionError(f"hazard: PV{grp}({g}) finds P of {self.P[grp]}")
+                if self.V[sv] != g:
+                    raise AssertionError(f"hazard: PV{grp}({g}) reads V stage {sv} holding tile {self.V[sv]}")
+                self.P_busy[grp] += 1
+                self.O_busy[grp] += 1
+
+                def pv_done(s=sv, g=g):
+                    self.P_busy[grp] -= 1
+                    self.O_busy[grp] -= 1
+                    if self.V[s] != g:
+                        raise AssertionError(f"hazard: V stage {s} overwritten during PV({g})")
+                    self.B[f"vempty{s}"].arrive()
+                    self.B[f"pvdone{grp}"].arrive()
+                self.later(pv_done)
+
+            def final_commit():
+                if self.O_busy[grp]:
+                    self.later(final_commit)
+                else:
+                    self.B["ofinal"].arrive()
+            self.later(final_commit)
+            yield ("sync",)
+            base += T
+            self.advance(bb, T)
+
+    def smem_softmax(self, grp):
+        base, bb = 0, [0, 0]
+        for u, T in enumerate(self.plan):
+            if self.route_in_kernel:
+                yield ("wait", "q", u)
+            if grp == 0:
+                self.B["list"].arrive()
+            else:
+                yield ("wait", "list", u)
+            for t in range(grp, T, 2):
+                g = base + t
+                _, use = self.buffer_of(g, t, bb)
+                yield ("wait", f"sfull{grp}", use)
+                if self.S[grp] is None or self.S[grp][:2] != ("S", g):
+                    raise AssertionError(f"hazard: softmax{grp}({g}) finds {self.S[grp]} in S{grp}")
+                if t >= 2 and self.mut != "p_skips_pvdone":
+                    yield ("wait", f"pvdone{grp}", use - 1)
+                self.S_read[grp] = g
+                self.B[f"sfree{grp}"].arrive()
+                # writes P and may rescale O: both must be at rest
+                if self.P_busy[grp]:
+                    raise AssertionError(f"hazard: softmax{grp}({g}) overwrites P while a PV reads it")
+                if self.O_busy[grp]:
+                    raise AssertionError(f"hazard: rescale of O{grp} at tile {g} with a PV in flight")
+                self.P[grp] = g
+                self.B[f"pfull{grp}{grp}"].arrive()
+            if T > 0:
+                yield ("wait", "ofinal", u)
+                if any(self.O_busy):
+                    raise AssertionError("hazard: the epilogue reads O with a PV in flight")
             yield ("sync",)
             base += T
             self.advance(bb, T)
