@@ -49,15 +49,19 @@ class Protocol:
         self.group_issuers = schedule == "group_issuers"
         self.smem_p = schedule == "smem_p"
         self.dephase = schedule == "split_dephase"
+        self.single = schedule == "split_single_issuer"
         self.rng = random.Random(seed)
         self.now, self.seq, self.events = 0, 0, []
-        if self.alt:  # one PV per tile: the owning group's
+        if schedule == "split_single_issuer":
+            pv_count, v_count = 1, 1
+        elif self.alt:  # one PV per tile: the owning group's
             pv_count = 2 if mutation == "alt_pvdone_count_2" else 1
             v_count = 1
         else:
             pv_count = 1 if mutation == "pvdone_count_1" else 2
             v_count = 2
-        self.B = {"q": Bar("q", 1), "ofinal": Bar("ofinal", 2), "list": Bar("list", 1)}
+        self.B = {"q": Bar("q", 1), "ofinal": Bar("ofinal", 1 if schedule == "split_single_issuer" else 2),
+                  "list": Bar("list", 1)}
         for s in range(nk):
             self.B[f"kfull{s}"], self.B[f"kempty{s}"] = Bar(f"kfull{s}", 1), Bar(f"kempty{s}", 1)
         for s in range(nv):
@@ -99,7 +103,10 @@ class Protocol:
         self.events.append((self.now + self.rng.choice([1, 2, 5, 20, 60]), self.seq, fn))
 
     def run(self):
-        if self.dephase:
+        if self.single:
+            roles = {"producer": self.producer(), "mma": self.single_issuer(),
+                     "sm0": self.softmax(0), "sm1": self.softmax(1)}
+        elif self.dephase:
             roles = {"producer": self.producer(), "qk": self.dephase_qk(), "pv0": self.dephase_pv(0),
                      "pv1": self.dephase_pv(1), "sm0": self.dephase_softmax(0), "sm1": self.dephase_softmax(1)}
         elif self.smem_p:
@@ -307,6 +314,70 @@ class Protocol:
             yield ("sync",)
             base += T
             self.advance(bb, T)
+
+    # ---- split columns, one thread issuing every product; its MMAs complete in issue order
+    def in_order(self, fn):
+        """Schedule an MMA completion no earlier than the previous MMA of the same thread."""
+        self.seq += 1
+        when = max(self.now + self.rng.choice([1, 2, 5, 20, 60]), getattr(self, "last_mma", 0))
+        self.last_mma = when
+        self.events.append((when, self.seq, fn))
+
+    def single_issuer(self):
+        base = 0
+        for u, T in enumerate(self.plan):
+            yield ("wait", "list", u)
+            yield ("wait", "q", u)
+
+            def qk(t):
+                g = base + t
+                b, s = g & 1, g % self.nk
+                yield ("wait", f"kfull{s}", g // self.nk)
+                if self.K[s] != g:
+                    raise AssertionError(f"hazard: QK({g}) reads K stage {s} holding tile {self.K[s]}")
+                self.S_busy[b].add(("QK", g))
+
+                def qk_done(b=b, s=s, g=g):
+                    # in issue order, every PV that read the previous P of S[b] has completed
+                    if any(x[0] == "PV" for x in self.S_busy[b]):
+                        raise AssertionError(f"hazard: QK({g}) wrote S{b} while a PV still read it")
+                    self.S_busy[b].discard(("QK", g))
+                    self.S[b] = ("S", g, False)
+                    self.B[f"sfull{b}"].arrive()
+                    self.B[f"kempty{s}"].arrive()
+                self.in_order(qk_done)
+            for t in range(min(T, 2)):
+                yield from qk(t)
+            for t in range(T):
+                g = base + t
+                b, s = g & 1, g % self.nv
+                yield ("wait", f"vfull{s}", g // self.nv)
+                for grp in range(2):
+                    yield ("wait", f"pfull{b}{grp}", g >> 1)
+                    if self.S[b] is None or self.S[b][:2] != ("P", g):
+                        raise AssertionError(f"hazard: PV{grp}({g}) finds {self.S[b]} in S{b}")
+                    self.S_busy[b].add(("PV", g, grp))
+                    self.O_busy[grp] += 1
+
+                    def pv_done(b=b, g=g, grp=grp):
+                        self.S_busy[b].discard(("PV", g, grp))
+                        self.O_busy[grp] -= 1
+                    self.in_order(pv_done)
+                if self.V[s] != g:
+                    raise AssertionError(f"hazard: PV({g}) reads V stage {s} holding tile {self.V[s]}")
+
+                def commit(b=b, s=s, g=g):
+                    if self.V[s] != g:
+                        raise AssertionError(f"hazard: V stage {s} overwritten during PV({g})")
+                    self.S[b] = ("P", g, True)
+                    self.B[f"vempty{s}"].arrive()
+                    self.B[f"pvdone{b}"].arrive()
+                self.in_order(commit)
+                if t + 2 < T:
+                    yield from qk(t + 2)
+            self.in_order(lambda: self.B["ofinal"].arrive())
+            yield ("sync",)
+            base += T
 
     # ---- split columns, P in shared memory, group 1 a phase behind
     def dephase_qk(self):

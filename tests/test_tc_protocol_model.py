@@ -14,7 +14,8 @@ import pytest
 from tc_protocol_model import Protocol, random_plan
 
 
-@pytest.mark.parametrize("schedule", ["split_dephase", "smem_p", "group_issuers", "alternate", "split"])
+@pytest.mark.parametrize("schedule", ["split_single_issuer", "split_dephase", "smem_p", "group_issuers",
+                                      "alternate", "split"])
 @pytest.mark.parametrize("nk,nv", [(3, 2), (4, 4)])  # d = 128 and d = 64 ring depths
 @pytest.mark.parametrize("route_in_kernel", [False, True])  # keep bits from the routing pass, or routed in place
 def test_protocol_has_no_deadlock_stale_wait_or_hazard(nk, nv, route_in_kernel, schedule):
@@ -30,6 +31,7 @@ def test_protocol_has_no_deadlock_stale_wait_or_hazard(nk, nv, route_in_kernel, 
     ("group_issuers", "vempty_one_back"),
     ("smem_p", "qk_skips_sfree"), ("smem_p", "p_skips_pvdone"), ("smem_p", "vempty_one_back"),
     ("split_dephase", "qk_skips_sfree"), ("split_dephase", "p_skips_pvdone"), ("split_dephase", "vempty_one_back"),
+    ("split_single_issuer", "vempty_one_back"),
 ])
 def test_planted_protocol_mistakes_are_caught(schedule, mutation):
     rng = random.Random(5)
