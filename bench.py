@@ -229,10 +229,12 @@ def oracle_sample(w, tau, budget_s: float, max_units: int = CPU_SAMPLE_UNITS, se
     return kept_tiles, elapsed, done, threads
 
 
-def measure_qknorm_rope_pool(w, Q, K, V, stream, pk, cpu_ok, max_over_ranks, barrier, world):
+def measure_qknorm_rope_pool(w, Q, K, V, stream, pk, cpu_ok, max_over_ranks, barrier, world, tau=None):
     """The fused QK-norm + RoPE + pooling step on the workload's own Q, K, V (standing in for the
     raw projections): CUDA-event time of the kernel alone, HBM roofline, and the oracle timed on a
-    bounded host sample."""
+    bounded host sample. With `tau`, also the pass that writes the query-block means, and the
+    forward on the pass's outputs with those means given (sol_attn_fwd_qbar) against the same
+    forward forming them from Q (sol_attn_fwd)."""
     import torch
     from block_sparse_attention_41_b200 import sol_attn as sa
     d, blk, nb = w.d, w.block, w.n_blocks
@@ -269,6 +271,65 @@ def measure_qknorm_rope_pool(w, Q, K, V, stream, pk, cpu_ok, max_over_ranks, bar
            "unfused_bytes": alg + elem_bytes, "GB/s": world * gbs, "bound": "hbm", "peak_GB/s": pk["hbm_gbs"],
            "frac": gbs / pk["hbm_gbs"],
            "note": "norm+RoPE then a separate pool would read the stored keys once more (unfused_bytes)"}
+    if tau is not None:
+        qb = torch.empty((w.B, w.H, nb, d), dtype=torch.float32, device=dev)
+
+        def run_q():
+            sa.sol_attn_qknorm_rope_pool(Q, K, V, tq, tk, tc, ts, blk, 1e-6, Qo, Ko, kb, vb, kl, vl, stream=stream,
+                                         qbar=qb)
+
+        def timed(fn, n):
+            for _ in range(2):
+                fn()
+            torch.cuda.synchronize()
+            barrier()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(n):
+                fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            return max_over_ranks(a.elapsed_time(b)) / n
+
+        ms_q = timed(run_q, n_it)
+        out["ms_with_qbar"] = ms_q
+        out["qbar_bytes"] = w.B * w.H * nb * d * 4
+        out["frac_with_qbar"] = (alg + out["qbar_bytes"]) / (ms_q * 1e-3) / 1e9 / pk["hbm_gbs"]
+        # the forward on the workload's own inputs with the query-block means given (formed here by
+        # torch from the same Q, standing in for the pass's output) against forming them in the
+        # routing pass, at the timed thresholds
+        kb2, vb2, kl2, vl2 = sa.sol_attn_pool(K, V, blk, stream=stream)
+        pad = nb * blk - w.L
+        qsum = torch.nn.functional.pad(Q.float(), (0, 0, 0, pad)).view(w.B, w.H, nb, blk, d).sum(3)
+        rows = torch.full((nb,), float(blk), device=dev)
+        rows[-1] = float(w.L - (nb - 1) * blk)
+        qb.copy_(qsum / rows.view(1, 1, nb, 1))
+        del qsum
+        Ofw = torch.empty_like(Q)
+        wsq = sa.new_workspace(w.B, w.H, w.L, blk, dev)
+        calls = {"own": lambda: sa.sol_attn_fwd(Q, K, V, kb2, vb2, kl2, vl2, tau, blk, blk, n_force=w.n_force, O=Ofw,
+                                                workspace=wsq, stream=stream),
+                 "given": lambda: sa.sol_attn_fwd_qbar(Q, K, V, kb2, vb2, kl2, vl2, qb, tau, n_force=w.n_force, O=Ofw,
+                                                       workspace=wsq, stream=stream)}
+        # interleaved one call at a time, so that clock drift under the power cap hits both alike
+        got = {"own": [], "given": []}
+        for it in range(12):
+            for name, fn in calls.items():
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                torch.cuda.synchronize()
+                if it >= 2:
+                    got[name].append(a.elapsed_time(b))
+        own, given = (max_over_ranks(statistics.median(got[k])) for k in ("own", "given"))
+        sa.sol_attn_check_device_error(wsq, stream)
+        out["forward_with_given_qbar"] = {
+            "fwd_ms_forming_qbar": own, "fwd_ms_given_qbar": given, "saved_ms": own - given,
+            "note": "the workload's inputs at the timed thresholds, median of 10 interleaved calls each; the "
+                    "given means spare the routing pass its read of Q"}
+        del kb2, vb2, kl2, vl2
+        del qb, Ofw, wsq
     del Qo, Ko, kb, vb, kl, vl
     if cpu_ok:
         import oracle
@@ -628,7 +689,7 @@ def run_ours(args, w):
     if not args.no_next and w.dtype == "bf16" and w.n_text == 0:
         next_rows = {"qknorm_rope_pool": measure_qknorm_rope_pool(
             w, Q, K, V, stream, pk, rank == 0 and world == 1 and not args.no_cpu_baseline, max_over_ranks, barrier,
-            world)}
+            world, tau=tau if w.block == 128 else None)}
         if w.d == 128:
             step(tau)  # the sweep left another density's output in O
             torch.cuda.synchronize()

@@ -44,6 +44,8 @@ struct FwdArgs {
   unsigned long long* cta_times = nullptr;  // measurement hook: [2 * cta_capacity] start/finish ns
   int cta_capacity = 0;
   const Qk8Operands* qk8 = nullptr;  // bf16 path: int8 Q, K and pooled keys for QK^T, or null
+  const float* qbar_in = nullptr;    // routing pass: fp32 [B*H, N_qb, d] query-block means given by the
+                                     // caller (the QK-norm + RoPE pass); null = computed from Q
 };
 
 cudaError_t launch_pool(const void* K, const void* V, bool bf16, int BH, int L, int d, int block,
@@ -64,6 +66,7 @@ struct RopePoolArgs {
   float* vbar;
   void* kbar_lp;  // bf16 [BH, N_kb, d]
   void* vbar_lp;
+  float* qbar = nullptr;  // out, optional: fp32 [BH, N_kb, d] means of the stored query rows per block
   int BH, L, d, block;
 };
 

@@ -7,11 +7,15 @@
 //   y'  = pairs (y_2i, y_2i+1) turned by the angle of cos/sin[t, i]
 // and the rotated rows are stored in bf16. The same pass sums the stored (bf16-rounded) keys and
 // the values of the block into the pooled vectors the sparse attention routes and corrects with,
-// so the keys are not read back from HBM by a separate pooling pass.
+// so the keys are not read back from HBM by a separate pooling pass. Optionally it also writes the
+// mean of the block's stored query rows (q_bar, the routing proxy's query side), so the routing
+// pass need not read Q again either.
 //
 // Layout: a lane owns 8 consecutive columns (16 bytes, four whole pairs) of one row; D/8 lanes
 // cover a row, so a warp covers 32 / (D/8) rows at once and the row's sum of squares is reduced
-// over those lanes only. HBM-bound: every byte is read or written once.
+// over those lanes only. HBM-bound: every byte is read or written once. The grid runs the heads
+// of one token range next to each other (head = blockIdx.x), so the cos/sin rows of that range
+// come from L2 for all but the first head.
 #include <cmath>
 
 #include "device_common.cuh"
@@ -39,6 +43,7 @@ struct RopePoolParams {
   float* vbar;             // [BH, nkb, D]
   __nv_bfloat16* kbar_lp;  // [BH, nkb, D]
   __nv_bfloat16* vbar_lp;  // [BH, nkb, D]
+  float* qbar;             // [BH, nkb, D] query-block means, or null
   int L, nkb, block;
   float eps;
 };
@@ -88,23 +93,23 @@ __global__ void __launch_bounds__(kThreads) sol_qknorm_rope_pool_kernel(const __
   constexpr int LPR = D / 8;          // lanes per row
   constexpr int RPW = 32 / LPR;       // rows per warp step
   constexpr int RG = kWarps * RPW;    // row groups per CTA
-  __shared__ float s_part[2][RG][D];  // per row group partial sums of the stored keys / the values
+  __shared__ float s_part[3][RG][D];  // per row group partial sums of the stored keys / the values / the stored queries
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.y;
+  const int bh = blockIdx.x;
   const int cl = lane % LPR, sub = lane / LPR;
   const int c0 = cl * 8;
   const int rg = warp * RPW + sub;
   const float inv_d = 1.0f / static_cast<float>(D);
-  const int jb_end = min(p.nkb, (static_cast<int>(blockIdx.x) + 1) * kBlocksPerCta);
-  for (int jb = blockIdx.x * kBlocksPerCta; jb < jb_end; ++jb) {
+  const int jb_end = min(p.nkb, (static_cast<int>(blockIdx.y) + 1) * kBlocksPerCta);
+  for (int jb = blockIdx.y * kBlocksPerCta; jb < jb_end; ++jb) {
     const int row0 = jb * p.block;
     const int n = min(p.block, p.L - row0);
     const size_t base = (static_cast<size_t>(bh) * p.L + row0) * D + c0;
 
-    float ak[8], av[8];
+    float ak[8], av[8], aq[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) ak[k] = av[k] = 0.f;
+    for (int k = 0; k < 8; ++k) ak[k] = av[k] = aq[k] = 0.f;
     // the loop runs the same number of times in every lane of a warp (the norm's shuffles need the
     // whole warp); lanes past the block's last row carry zeros and store nothing
     for (int rbase = warp * RPW; rbase < n; rbase += RG) {
@@ -126,6 +131,7 @@ __global__ void __launch_bounds__(kThreads) sol_qknorm_rope_pool_kernel(const __
         for (int k = 0; k < 8; ++k) {
           ak[k] += xk[k];
           av[k] += xv[k];
+          aq[k] += xq[k];
         }
       }
     }
@@ -133,11 +139,13 @@ __global__ void __launch_bounds__(kThreads) sol_qknorm_rope_pool_kernel(const __
     for (int k = 0; k < 8; ++k) {
       s_part[0][rg][c0 + k] = ak[k];
       s_part[1][rg][c0 + k] = av[k];
+      s_part[2][rg][c0 + k] = aq[k];
     }
     __syncthreads();
-    // thread t < 2 D: column t % D of the keys (t < D) or the values
-    if (tid < 2 * D) {
-      const int which = tid / D, c = tid % D;
+    // index i < 3 D: column i % D of the keys, the values or the queries (i / D = 0, 1, 2)
+    const int nsum = p.qbar != nullptr ? 3 * D : 2 * D;
+    for (int i = tid; i < nsum; i += kThreads) {
+      const int which = i / D, c = i % D;
       float sum = 0.f;
 #pragma unroll 4
       for (int k = 0; k < RG; ++k) sum += s_part[which][k][c];
@@ -146,9 +154,11 @@ __global__ void __launch_bounds__(kThreads) sol_qknorm_rope_pool_kernel(const __
       if (which == 0) {
         p.kbar[o] = mean;
         p.kbar_lp[o] = __float2bfloat16_rn(mean);
-      } else {
+      } else if (which == 1) {
         p.vbar[o] = mean;
         p.vbar_lp[o] = __float2bfloat16_rn(mean);
+      } else {
+        p.qbar[o] = mean;
       }
     }
     __syncthreads();  // s_part is reused by the next block
@@ -171,11 +181,12 @@ cudaError_t launch_t(const RopePoolArgs& a, cudaStream_t stream) {
   p.vbar = a.vbar;
   p.kbar_lp = static_cast<__nv_bfloat16*>(a.kbar_lp);
   p.vbar_lp = static_cast<__nv_bfloat16*>(a.vbar_lp);
+  p.qbar = a.qbar;
   p.L = a.L;
   p.block = a.block;
   p.nkb = (a.L + a.block - 1) / a.block;
   p.eps = a.eps;
-  const dim3 grid((p.nkb + kBlocksPerCta - 1) / kBlocksPerCta, a.BH);
+  const dim3 grid(a.BH, (p.nkb + kBlocksPerCta - 1) / kBlocksPerCta);
   sol_qknorm_rope_pool_kernel<D><<<grid, kThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }

@@ -328,7 +328,7 @@ __global__ void __launch_bounds__(kRouteThreads) sol_route_kernel(const __grid_c
 template <int D, int R>
 cudaError_t launch_route_t(const FwdArgs& a, cudaStream_t stream) {
   RouteParams p;
-  p.qbar = a.route_qbar;
+  p.qbar = a.qbar_in != nullptr ? a.qbar_in : a.route_qbar;
   p.kbar = a.kbar;
   p.bits = a.route_bits;
   p.kept_mask = a.kept_mask;
@@ -343,11 +343,14 @@ cudaError_t launch_route_t(const FwdArgs& a, cudaStream_t stream) {
   p.k_keep = a.k_keep;
   p.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   for (int h = 0; h < kMaxHeads; ++h) p.tau[h] = h < a.H ? a.tau[h] : 0.f;
-  constexpr int QB = 2;
-  sol_qbar_kernel<D, QB><<<dim3((p.nqb + QB - 1) / QB, p.BH), kRouteThreads, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(a.Q), a.route_qbar, p.L, p.nqb);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (a.qbar_in == nullptr) {  // else the caller's means, from the pass that stored Q
+    constexpr int QB = 2;
+    sol_qbar_kernel<D, QB><<<dim3((p.nqb + QB - 1) / QB, p.BH), kRouteThreads, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(a.Q), a.route_qbar, p.L, p.nqb);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   const size_t smem = (static_cast<size_t>(R) * D + static_cast<size_t>(R) * p.nkb) * sizeof(float);
   e = cudaFuncSetAttribute(sol_route_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;

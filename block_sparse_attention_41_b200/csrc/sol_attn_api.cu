@@ -228,10 +228,12 @@ sol_status sol_attn_pool(const void* K, const void* V, sol_dtype dt, int B, int 
   return SOL_OK;
 }
 
-sol_status sol_attn_qknorm_rope_pool(const void* Q, const void* K, const void* V, const float* gain_q,
-                                     const float* gain_k, const float* rope_cos, const float* rope_sin, float eps,
-                                     int B, int H, int L, int d, int block_k, void* Q_out, void* K_out, float* kbar,
-                                     float* vbar, void* kbar_lp, void* vbar_lp, void* stream) {
+// The QK-norm + RoPE + pooling pass; qbar (optional) receives the query-block means.
+static sol_status qknorm_rope_pool_impl(const void* Q, const void* K, const void* V, const float* gain_q,
+                                        const float* gain_k, const float* rope_cos, const float* rope_sin, float eps,
+                                        int B, int H, int L, int d, int block_k, void* Q_out, void* K_out,
+                                        float* kbar, float* vbar, void* kbar_lp, void* vbar_lp, float* qbar,
+                                        void* stream) {
   g_last_error.clear();
   if (!size_ok(B, 1 << 16) || !size_ok(H, 1 << 16) || !size_ok(L, 1 << 28) || !size_ok(d, 1 << 16) ||
       !size_ok(block_k, 1 << 20))
@@ -245,6 +247,9 @@ sol_status sol_attn_qknorm_rope_pool(const void* Q, const void* K, const void* V
   if (d != 64 && d != 128) return fail(SOL_EUNSUPPORTED, "QK-norm + RoPE + pooling needs d in {64, 128} (d=%d)", d);
   if (block_k > 4096) return fail(SOL_EUNSUPPORTED, "block_k must be <= 4096");
   if (static_cast<long long>(B) * H > 65535) return fail(SOL_EUNSUPPORTED, "B*H must be <= 65535");
+  // the grid's second dimension runs over groups of 4 key blocks
+  if ((static_cast<long long>(L) + block_k - 1) / block_k > 4ll * 65535)
+    return fail(SOL_EUNSUPPORTED, "ceil(L / block_k) must be <= %d", 4 * 65535);
   int sms = 0;
   sol_status st = current_device(&sms);
   if (st != SOL_OK) return st;
@@ -263,6 +268,7 @@ sol_status sol_attn_qknorm_rope_pool(const void* Q, const void* K, const void* V
   a.vbar = vbar;
   a.kbar_lp = kbar_lp;
   a.vbar_lp = vbar_lp;
+  a.qbar = qbar;
   a.BH = B * H;
   a.L = L;
   a.d = d;
@@ -270,6 +276,27 @@ sol_status sol_attn_qknorm_rope_pool(const void* Q, const void* K, const void* V
   cudaError_t e = sol::launch_qknorm_rope_pool(a, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "QK-norm + RoPE + pooling launch");
   return SOL_OK;
+}
+
+sol_status sol_attn_qknorm_rope_pool(const void* Q, const void* K, const void* V, const float* gain_q,
+                                     const float* gain_k, const float* rope_cos, const float* rope_sin, float eps,
+                                     int B, int H, int L, int d, int block_k, void* Q_out, void* K_out, float* kbar,
+                                     float* vbar, void* kbar_lp, void* vbar_lp, void* stream) {
+  return qknorm_rope_pool_impl(Q, K, V, gain_q, gain_k, rope_cos, rope_sin, eps, B, H, L, d, block_k, Q_out, K_out,
+                               kbar, vbar, kbar_lp, vbar_lp, nullptr, stream);
+}
+
+sol_status sol_attn_qknorm_rope_pool_qbar(const void* Q, const void* K, const void* V, const float* gain_q,
+                                          const float* gain_k, const float* rope_cos, const float* rope_sin,
+                                          float eps, int B, int H, int L, int d, int block_k, void* Q_out,
+                                          void* K_out, float* kbar, float* vbar, void* kbar_lp, void* vbar_lp,
+                                          float* qbar, void* stream) {
+  if (qbar == nullptr || !aligned16(qbar)) {
+    g_last_error.clear();
+    return fail(SOL_EINVAL, "qbar must be a non-null, 16-byte aligned device pointer");
+  }
+  return qknorm_rope_pool_impl(Q, K, V, gain_q, gain_k, rope_cos, rope_sin, eps, B, H, L, d, block_k, Q_out, K_out,
+                               kbar, vbar, kbar_lp, vbar_lp, qbar, stream);
 }
 
 sol_status sol_attn_quantize_qk8(const void* Q, const void* K, const float* kbar, int B, int H, int L, int d,
@@ -323,7 +350,7 @@ sol_status fwd_impl(const void* Q, const void* K, const void* V, const float* kb
                     const void* kbar_lp, const void* vbar_lp, const float* tau, sol_dtype dt, int B, int H, int L,
                     int d, int block_q, int block_k, int n_force, void* O, uint8_t* kept_mask, float* density,
                     void* workspace, size_t ws_bytes, void* stream, int k_keep,
-                    const sol::Qk8Operands* qk8 = nullptr) {
+                    const sol::Qk8Operands* qk8 = nullptr, const float* qbar_in = nullptr) {
   if (dt != SOL_F32 && dt != SOL_BF16) return fail(SOL_EINVAL, "unknown dtype %d", static_cast<int>(dt));
   if (!size_ok(B, 1 << 16) || !size_ok(H, 1 << 16) || !size_ok(L, 1 << 28) || !size_ok(d, 1 << 16) ||
       !size_ok(block_q, 1 << 20) || !size_ok(block_k, 1 << 20))
@@ -419,6 +446,7 @@ sol_status fwd_impl(const void* Q, const void* K, const void* V, const float* kb
     if ((st = make_map(&maps[3], i8 ? qk8->kb8 : kbar_lp, d, nkb_i, B * H, i8)) != SOL_OK) return st;
     if ((st = make_map(&maps[4], vbar_lp, d, nkb_i, B * H)) != SOL_OK) return st;
     a.qk8 = qk8;
+    a.qbar_in = route_pass ? qbar_in : nullptr;
     if (route_pass) {
       e = sol::launch_route(a, s);
       if (e != cudaSuccess) return cuda_fail(e, "routing launch");
@@ -458,6 +486,19 @@ sol_status sol_attn_fwd_topk(const void* Q, const void* K, const void* V, const 
   float zeros[sol::kMaxHeads] = {};  // unused by the routing pass in this mode; valid thresholds
   return fwd_impl(Q, K, V, kbar, nullptr, kbar_lp, vbar_lp, zeros, SOL_BF16, B, H, L, d, 128, 128, n_force, O,
                   kept_mask, density, workspace, ws_bytes, stream, k_keep);
+}
+
+sol_status sol_attn_fwd_qbar(const void* Q, const void* K, const void* V, const float* kbar, const float* vbar,
+                             const void* kbar_lp, const void* vbar_lp, const float* qbar, const float* tau, int B,
+                             int H, int L, int d, int n_force, void* O, uint8_t* kept_mask, float* density,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  if (B < 1 || H < 1 || L < 1) return fail(SOL_EINVAL, "sizes must be positive (B=%d H=%d L=%d)", B, H, L);
+  if (qbar == nullptr || !aligned16(qbar)) return fail(SOL_EINVAL, "qbar must be a non-null, 16-byte aligned device pointer");
+  if (workspace == nullptr || ws_bytes < sol_attn_fwd_workspace_bytes(B, H, L, 128))
+    return fail(SOL_EINVAL, "the given query-block means feed the routing pass, which needs the full workspace");
+  return fwd_impl(Q, K, V, kbar, vbar, kbar_lp, vbar_lp, tau, SOL_BF16, B, H, L, d, 128, 128, n_force, O, kept_mask,
+                  density, workspace, ws_bytes, stream, 0, nullptr, qbar);
 }
 
 sol_status sol_attn_fwd_qk8(const void* Q, const int8_t* q8, const int8_t* k8, const int8_t* kbar8,

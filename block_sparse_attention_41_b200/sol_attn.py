@@ -37,6 +37,8 @@ EXPORTED = (
     "sol_attn_fwd_topk",
     "sol_attn_quantize_qk8",
     "sol_attn_fwd_qk8",
+    "sol_attn_qknorm_rope_pool_qbar",
+    "sol_attn_fwd_qbar",
 )
 
 
@@ -79,6 +81,12 @@ def load_library() -> ctypes.CDLL:
     lib.sol_attn_qknorm_rope_pool.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, i32, i32, i32, i32,
                                               vp, vp, vp, vp, vp, vp, vp]
     lib.sol_attn_qknorm_rope_pool.restype = i32
+    lib.sol_attn_qknorm_rope_pool_qbar.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, i32, i32, i32,
+                                                   i32, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.sol_attn_qknorm_rope_pool_qbar.restype = i32
+    lib.sol_attn_fwd_qbar.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, f32p, i32, i32, i32, i32, i32, vp, vp, vp, vp,
+                                      ctypes.c_size_t, vp]
+    lib.sol_attn_fwd_qbar.restype = i32
     lib.sol_attn_quantize_qk8.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.sol_attn_quantize_qk8.restype = i32
     lib.sol_attn_fwd_qk8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, f32p, i32, i32, i32, i32, i32, vp, vp,
@@ -168,10 +176,12 @@ def sol_attn_pool(K: torch.Tensor, V: torch.Tensor, block_k: int, kbar=None, vba
 
 
 def sol_attn_qknorm_rope_pool(Q, K, V, gain_q, gain_k, rope_cos, rope_sin, block_k: int, eps: float = 1e-6,
-                              Q_out=None, K_out=None, kbar=None, vbar=None, kbar_lp=None, vbar_lp=None, stream=None):
+                              Q_out=None, K_out=None, kbar=None, vbar=None, kbar_lp=None, vbar_lp=None, stream=None,
+                              qbar=None, want_qbar: bool = False):
     """QK RMS norm + rotary embedding of Q and K, and the block means of the stored K and of V, in
-    one pass. Returns (Q_out, K_out, kbar, vbar, kbar_lp, vbar_lp). Pass Q_out=Q, K_out=K to
-    work in place."""
+    one pass. Returns (Q_out, K_out, kbar, vbar, kbar_lp, vbar_lp), plus qbar (the block means of
+    the stored Q, for sol_attn_fwd_qbar) when want_qbar or a qbar tensor is given. Pass Q_out=Q,
+    K_out=K to work in place."""
     for n, t in (("Q", Q), ("K", K), ("V", V)):
         _need_cuda(n, t, torch.bfloat16)
     B, H, L, d = Q.shape
@@ -189,12 +199,21 @@ def sol_attn_qknorm_rope_pool(Q, K, V, gain_q, gain_k, rope_cos, rope_sin, block
     vbar = torch.empty((B, H, nkb, d), dtype=torch.float32, device=dev) if vbar is None else vbar
     kbar_lp = torch.empty((B, H, nkb, d), dtype=torch.bfloat16, device=dev) if kbar_lp is None else kbar_lp
     vbar_lp = torch.empty((B, H, nkb, d), dtype=torch.bfloat16, device=dev) if vbar_lp is None else vbar_lp
-    st = load_library().sol_attn_qknorm_rope_pool(
+    if qbar is None and not want_qbar:
+        st = load_library().sol_attn_qknorm_rope_pool(
+            _ptr(Q), _ptr(K), _ptr(V), _ptr(gain_q), _ptr(gain_k), _ptr(rope_cos), _ptr(rope_sin),
+            ctypes.c_float(eps), B, H, L, d, block_k, _ptr(Q_out), _ptr(K_out), _ptr(kbar), _ptr(vbar), _ptr(kbar_lp),
+            _ptr(vbar_lp), _stream(stream))
+        _check(st, "sol_attn_qknorm_rope_pool")
+        return Q_out, K_out, kbar, vbar, kbar_lp, vbar_lp
+    qbar = torch.empty((B, H, nkb, d), dtype=torch.float32, device=dev) if qbar is None else qbar
+    _need_cuda("qbar", qbar, torch.float32)
+    st = load_library().sol_attn_qknorm_rope_pool_qbar(
         _ptr(Q), _ptr(K), _ptr(V), _ptr(gain_q), _ptr(gain_k), _ptr(rope_cos), _ptr(rope_sin), ctypes.c_float(eps),
         B, H, L, d, block_k, _ptr(Q_out), _ptr(K_out), _ptr(kbar), _ptr(vbar), _ptr(kbar_lp), _ptr(vbar_lp),
-        _stream(stream))
-    _check(st, "sol_attn_qknorm_rope_pool")
-    return Q_out, K_out, kbar, vbar, kbar_lp, vbar_lp
+        _ptr(qbar), _stream(stream))
+    _check(st, "sol_attn_qknorm_rope_pool_qbar")
+    return Q_out, K_out, kbar, vbar, kbar_lp, vbar_lp, qbar
 
 
 def sol_attn_quantize_qk8(Q, K, kbar, stream=None):
@@ -330,6 +349,35 @@ def sol_attn_fwd_topk(Q, K, V, kbar, kbar_lp, vbar_lp, k_keep: int, n_force: int
         _ptr(Q), _ptr(K), _ptr(V), _ptr(kbar), _ptr(kbar_lp), _ptr(vbar_lp), int(k_keep), B, H, L, d, int(n_force),
         _ptr(O), _ptr(kept_mask), _ptr(density), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "sol_attn_fwd_topk")
+    return O
+
+
+def sol_attn_fwd_qbar(Q, K, V, kbar, vbar, kbar_lp, vbar_lp, qbar, tau, n_force: int = 0, O=None, kept_mask=None,
+                      density=None, workspace=None, stream=None):
+    """Fused forward whose routing pass takes the query-block means qbar (fp32 [B, H, N_qb, d],
+    from sol_attn_qknorm_rope_pool(..., want_qbar=True)) instead of reading Q for them (bf16,
+    blocks of 128). Returns O."""
+    _need_cuda("Q", Q, torch.bfloat16)
+    for n, t in (("K", K), ("V", V)):
+        _need_cuda(n, t, torch.bfloat16)
+    _need_cuda("qbar", qbar, torch.float32)
+    B, H, L, d = Q.shape
+    if K.shape != Q.shape or V.shape != Q.shape:
+        raise ValueError("Q, K and V must have the same shape [B, H, L, d]")
+    if tuple(qbar.shape) != (B, H, -(-L // 128), d):
+        raise ValueError("qbar must be [B, H, ceil(L/128), d]")
+    tau = [float(x) for x in tau]
+    if len(tau) != H:
+        raise ValueError(f"tau must hold H={H} values")
+    tau_arr = (ctypes.c_float * H)(*tau)
+    if O is None:
+        O = torch.empty_like(Q)
+    if workspace is None:
+        workspace = new_workspace(B, H, L, 128, Q.device)
+    st = load_library().sol_attn_fwd_qbar(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(kbar), _ptr(vbar), _ptr(kbar_lp), _ptr(vbar_lp), _ptr(qbar), tau_arr, B, H, L,
+        d, int(n_force), _ptr(O), _ptr(kept_mask), _ptr(density), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "sol_attn_fwd_qbar")
     return O
 
 

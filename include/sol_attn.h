@@ -105,6 +105,20 @@ sol_status sol_attn_qknorm_rope_pool(const void* Q, const void* K, const void* V
                                      void* K_out, float* kbar, float* vbar, void* kbar_lp, void* vbar_lp,
                                      void* stream);
 
+/* The same pass, also writing the query-block means the routing proxy needs (NEXT-1: the pages'
+ * "fused QK+RoPE" folds the pooling of Q into the pass that stores Q):
+ *   qbar   device, out, float32 [B, H, N_kb, d]: for each block of block_k rows, the mean of the
+ *          STORED (bf16-rounded) query rows Q_out, over the block's valid rows
+ * Pass it to sol_attn_fwd_qbar with block_k = 128, and the routing pass does not read Q again.
+ * Other arguments, limits and errors as for sol_attn_qknorm_rope_pool; qbar non-null and 16-byte
+ * aligned, else SOL_EINVAL. */
+sol_status sol_attn_qknorm_rope_pool_qbar(const void* Q, const void* K, const void* V,
+                                          const float* gain_q, const float* gain_k,
+                                          const float* rope_cos, const float* rope_sin, float eps, int B,
+                                          int H, int L, int d, int block_k, void* Q_out, void* K_out,
+                                          float* kbar, float* vbar, void* kbar_lp, void* vbar_lp,
+                                          float* qbar, void* stream);
+
 /* 8-bit operands of QK^T for sol_attn_fwd_qk8 (NEXT-2: the review page of the Sol Video Inference
  * Engine paper lists SageAttention's 8-bit attention with outlier smoothing; the Sol-Engine README
  * news reports fused 8-bit compute). From Q, K (bf16 [B, H, L, d]) and the fp32 pooled keys kbar
@@ -178,6 +192,20 @@ sol_status sol_attn_fwd_topk(const void* Q, const void* K, const void* V, const 
                              const void* kbar_lp, const void* vbar_lp, int k_keep, int B, int H, int L,
                              int d, int n_force, void* O, uint8_t* kept_mask, float* density,
                              void* workspace, size_t ws_bytes, void* stream);
+
+/* sol_attn_fwd with the query-block means given by the caller (qbar, fp32 [B, H, N_qb, d], as
+ * sol_attn_qknorm_rope_pool_qbar writes them for the Q it stores): the routing pass takes them
+ * instead of reading Q to form q_bar (Sol-Attn project page, Abstract: the proxy score pools the
+ * query block). The means may differ from the ones sol_attn_fwd forms in the last bits (another
+ * fp32 summation order), which can move a block whose proxy score lies within that rounding of
+ * the threshold. SOL_BF16 only, blocks of 128, d in {64, 128}; the workspace must have the full
+ * size of sol_attn_fwd_workspace_bytes. qbar non-null and 16-byte aligned, else SOL_EINVAL. Other
+ * arguments, limits and errors as for sol_attn_fwd. */
+sol_status sol_attn_fwd_qbar(const void* Q, const void* K, const void* V, const float* kbar,
+                             const float* vbar, const void* kbar_lp, const void* vbar_lp,
+                             const float* qbar, const float* tau, int B, int H, int L, int d,
+                             int n_force, void* O, uint8_t* kept_mask, float* density, void* workspace,
+                             size_t ws_bytes, void* stream);
 
 /* The forward with 8-bit QK^T (NEXT-2): the exact tiles' and the correction's scores come from the
  * int8 codes of sol_attn_quantize_qk8 (tcgen05 kind::i8, int32 accumulation), scaled by

@@ -123,6 +123,7 @@ def test_qknorm_rope_pool_rejects_invalid_arguments(lib):
     assert rope_pool(lib, d=96) == sa.SOL_EUNSUPPORTED
     assert rope_pool(lib, blk=8192) == sa.SOL_EUNSUPPORTED
     assert rope_pool(lib, B=300, H=300) == sa.SOL_EUNSUPPORTED
+    assert rope_pool(lib, L=4 * 65535 + 1, blk=1) == sa.SOL_EUNSUPPORTED  # the grid's second dimension
 
 
 def test_check_device_error_rejects_null(lib):
@@ -200,3 +201,24 @@ def test_topk_entry_rejects_invalid_arguments(lib):
     assert call(workspace=None) == sa.SOL_EINVAL
     assert call(L=0) == sa.SOL_EINVAL
     assert call(H=300) == sa.SOL_EUNSUPPORTED
+
+
+def test_qbar_entries_reject_invalid_arguments(lib):
+    tau = (ctypes.c_float * 2)(0.5, 0.5)
+
+    def fwd(qbar=P[9], ws=1 << 30, workspace=P[8], L=1000):
+        return lib.sol_attn_fwd_qbar(P[0], P[1], P[2], P[3], P[4], P[5], P[6], qbar, tau, 1, 2, L, 128, 0, P[7], None,
+                                     None, workspace, ws, None)
+    assert fwd(qbar=None) == sa.SOL_EINVAL
+    assert "qbar" in lib.sol_attn_last_error().decode()
+    assert fwd(qbar=ctypes.c_void_p(0x1008)) == sa.SOL_EINVAL  # not 16-byte aligned
+    assert fwd(ws=256) == sa.SOL_EINVAL
+    assert "full workspace" in lib.sol_attn_last_error().decode()
+    assert fwd(workspace=None) == sa.SOL_EINVAL
+    assert fwd(L=0) == sa.SOL_EINVAL
+
+    def pool(qbar=P[9]):
+        return lib.sol_attn_qknorm_rope_pool_qbar(P[0], P[1], P[2], P[3], P[4], P[5], P[6], ctypes.c_float(1e-6), 1, 2,
+                                                  1000, 128, 128, P[7], P[8], P[9], P[10], P[11], P[11], qbar, None)
+    assert pool(qbar=None) == sa.SOL_EINVAL
+    assert "qbar" in lib.sol_attn_last_error().decode()

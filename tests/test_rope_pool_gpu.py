@@ -114,3 +114,83 @@ def test_qknorm_rope_pool_full_720p_shape_sampled():
         got_k = kbar[0, h].double().cpu().numpy()[blocks]
         got_v = vbar[0, h].double().cpu().numpy()[blocks]
         assert np.max(np.abs(got_k - kb)) <= 1e-4 and np.max(np.abs(got_v - vb)) <= 1e-5
+
+
+# ------------------------------------------------------------------------------------------------
+# the query-block means written by the same pass, and the forward whose routing takes them
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("grid,d,blk", [((5, 10, 20), 128, 128), ((3, 7, 13), 64, 128), ((1, 1, 77), 64, 64)])
+def test_qbar_output_is_the_mean_of_the_stored_query_rows(grid, d, blk):
+    """q_bar is the mean of each block's stored (bf16) query rows over its valid rows; asking for it
+    changes no other output of the pass."""
+    B, H = 1, 3
+    L = grid[0] * grid[1] * grid[2]
+    rng = np.random.default_rng(L + 7 * d + blk)
+    Qh, Kh, Vh = (round_to_bf16(rng.standard_normal((B, H, L, d)) * s) for s in (2.0, 0.7, 1.0))
+    cos, sin = wl.rope_tables(grid, d)
+    gq, gk = wl.qk_norm_gains(d, L)
+    Q, K, V = (torch.from_numpy(x).to(torch.bfloat16).cuda() for x in (Qh, Kh, Vh))
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()  # noqa: E731
+    args = (Q, K, V, dev(gq), dev(gk), dev(cos), dev(sin), blk, EPS)
+    plain = sa.sol_attn_qknorm_rope_pool(*args)
+    withq = sa.sol_attn_qknorm_rope_pool(*args, want_qbar=True)
+    torch.cuda.synchronize()
+    assert len(withq) == 7
+    for a, b in zip(plain, withq[:6]):
+        assert torch.equal(a, b)
+    qbar = withq[6].double().cpu().numpy()
+    Qg = withq[0].double().cpu().numpy()
+    for h in range(H):
+        ref = oracle.pool_blocks(Qg[0, h], blk)  # the stored rows, pooled in float64
+        assert qbar[0, h].shape == ref.shape
+        assert np.max(np.abs(qbar[0, h] - ref)) <= 2e-6 * max(1.0, float(np.abs(Qg).max()))
+        # and against the means of the oracle's own stored rows: a difference of means is at most
+        # the mean of the row differences (the rare last-bit bf16 roundings), plus fp32 summation
+        Qr, _, _, _ = oracle.qknorm_rope_pool_head(Qh[0, h], Kh[0, h], Vh[0, h], gq, gk, cos, sin, EPS, blk, _bf16_64)
+        bound = oracle.pool_blocks(np.abs(Qg[0, h] - Qr), blk) + 2e-6 * max(1.0, float(np.abs(Qg).max()))
+        assert np.all(np.abs(qbar[0, h] - oracle.pool_blocks(Qr, blk)) <= bound)
+
+
+@pytest.mark.parametrize("L,d,tau,n_force", [(3000, 128, [0.4, 1.0], 0), (1111, 64, [0.0, 2.0], 2),
+                                             (16_500, 128, [0.6, 0.3], 0)])
+def test_forward_with_given_qbar_matches_the_oracle(L, d, tau, n_force):
+    """The pass's q_bar fed to sol_attn_fwd_qbar: the routing pass reads no Q, the kept sets meet
+    the oracle's routing acceptance, O is within the bf16 tolerance of the oracle, and the result
+    agrees with sol_attn_fwd on the same stored inputs (masks may differ only where the proxy score
+    lies within rounding of the threshold)."""
+    from test_parity_gpu import local_inputs, full_compare, check_bf16, check_mask_density, report
+    B, H = 1, 2
+    Qh, Kh, Vh = local_inputs(B, H, L, d, seed=L + d)
+    grid = (1, 1, L)
+    cos, sin = wl.rope_tables(grid, d)
+    gq, gk = wl.qk_norm_gains(d, L)
+    Q, K, V = (torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).cuda() for x in (Qh, Kh, Vh))
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()  # noqa: E731
+    Qs, Ks, kbar, vbar, klp, vlp, qbar = sa.sol_attn_qknorm_rope_pool(Q, K, V, dev(gq), dev(gk), dev(cos), dev(sin),
+                                                                      128, EPS, want_qbar=True)
+    nb = -(-L // 128)
+    masks, outs = [], []
+    for use_qbar in (True, False):
+        mask = torch.empty((B, H, nb, nb), dtype=torch.uint8, device="cuda")
+        dens = torch.empty((B, H), dtype=torch.float32, device="cuda")
+        ws = sa.new_workspace(B, H, L, 128, Q.device)
+        if use_qbar:
+            O = sa.sol_attn_fwd_qbar(Qs, Ks, V, kbar, vbar, klp, vlp, qbar, tau, n_force=n_force, kept_mask=mask,
+                                     density=dens, workspace=ws)
+        else:
+            O = sa.sol_attn_fwd(Qs, Ks, V, kbar, vbar, klp, vlp, tau, 128, 128, n_force=n_force, kept_mask=mask,
+                                density=dens, workspace=ws)
+        sa.sol_attn_check_device_error(ws)
+        check_mask_density(mask, dens, n_force)
+        masks.append(mask)
+        outs.append(O)
+    Qsh, Ksh = Qs.double().cpu().numpy(), Ks.double().cpu().numpy()
+    st = full_compare(Qsh, Ksh, Vh.astype(np.float64), outs[0], masks[0], tau, 128, n_force=n_force)
+    report(f"fwd with given q_bar L={L} d={d}", st)
+    check_bf16(st)
+    differ = int((masks[0] != masks[1]).sum())
+    assert differ <= st["band_entries"], (differ, st["band_entries"])
+    if differ == 0:
+        diff = (outs[0].double() - outs[1].double()).abs()
+        assert float(diff.max()) <= 2e-2 and float(diff.mean()) <= 2e-3
