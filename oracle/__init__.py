@@ -19,6 +19,15 @@ from .sol_attn_oracle import (  # noqa: F401
     unit_terms,
 )
 from .qknorm_rope_oracle import qknorm_rope_pool_head, rms_norm, rope  # noqa: F401
-from .mxfp8_oracle import forward_head_mx, int8_quantize_tiles, mx_quantize, no_quantize, round_e4m3  # noqa: F401,E501
+from .mxfp8_oracle import (  # noqa: F401
+    channel_scales,
+    e4m3_channel_quantize,
+    e4m3_plain,
+    forward_head_mx,
+    int8_quantize_tiles,
+    mx_quantize,
+    no_quantize,
+    round_e4m3,
+)
 from .topk_routing_oracle import forward_head_topk, keep_count, route_topk  # noqa: F401
 from .taylor_correction_oracle import cross_moments, forward_head_taylor, unit_forward_taylor  # noqa: F401

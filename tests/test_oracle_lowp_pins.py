@@ -186,6 +186,91 @@ def test_error_against_the_exact_definition_on_a_seeded_case():
     assert efp.mean() > e8.mean()
 
 
+# ---- the "e4m3_channel" PV reading: plain E4M3 weights, E4M3 values with one scale per channel ----
+
+def test_channel_scales_hand_example():
+    V = np.array([[896.0, 0.0, 0.25],
+                  [-3.0, 0.0, -1.0],
+                  [5.0, 0.0, 0.5]])
+    s = oracle.channel_scales(V)
+    assert np.array_equal(s, [2.0, 1.0, 1.0 / 448.0])  # amax / 448 per column; 1 for a zero column
+
+
+def test_e4m3_channel_quantize_hand_example():
+    s = np.array([2.0, 0.5])
+    x = np.array([[896.0, 224.0],    # 448 * s: the top code exactly
+                  [19.0, 4.5],       # 9.5 -> 9.5 is not E4M3 (8..16 step 1): tie -> 10 (even); 9 -> 9
+                  [-3.0, 0.0],       # -1.5 exact; 0 exact
+                  [2000.0, -500.0]])  # beyond 448 s: clamped to +-448 s
+    q = oracle.e4m3_channel_quantize(x, s)
+    assert np.array_equal(q, [[896.0, 224.0], [20.0, 4.5], [-3.0, 0.0], [896.0, -224.0]])
+    # channels are independent: changing channel 1 leaves channel 0 as it was
+    x2 = x.copy()
+    x2[:, 1] *= 3
+    assert np.array_equal(oracle.e4m3_channel_quantize(x2, s)[:, 0], q[:, 0])
+
+
+def _two_level_case(d=16, L=256):
+    """Identical queries; keys 0 in block 0 and e_0 in block 1, scaled so the log2-domain logits
+    are exactly 0 and 1; V integers with a 448 in every channel (exact E4M3, scale 1)."""
+    rng = np.random.default_rng(31)
+    q = np.zeros(d)
+    q[0] = math.sqrt(d) * math.log(2.0)
+    Q = np.tile(q, (L, 1))
+    K = np.zeros((L, d))
+    K[128:, 0] = 1.0
+    V = rng.integers(-7, 8, size=(L, d)).astype(np.float64)  # |v| <= 7: at most 3 significant bits
+    V[5] = 448.0
+    return Q, K, V
+
+
+def test_e4m3_channel_reading_is_exact_on_a_closed_form_case():
+    # weights 2^(0-1) = 0.5 for block 0 and 2^(1-1) = 1 for block 1, both exact in E4M3; values
+    # exact under their channel scales (amax 448 -> scale 1): the reading reproduces the definition
+    Q, K, V = _two_level_case()
+    O, keep = oracle.forward_head_mx(Q, K, V, math.inf, 128, qk="none", pv="e4m3_channel")
+    assert keep.all()
+    closed = (0.5 * V[:128].sum(axis=0) + V[128:].sum(axis=0)) / (0.5 * 128 + 128)
+    assert np.max(np.abs(O - closed[None, :])) <= 1e-12
+    ref, _, _, _ = oracle.forward_head(Q, K, V, math.inf, 128, 128, 0)
+    assert np.max(np.abs(O - ref)) <= 1e-12
+
+
+def test_e4m3_channel_values_take_the_channel_scale_and_pooled_values_take_v_scales():
+    # a column of V scaled by 2^k: its scale is 2^k times larger, so its codes and the output's
+    # column scale by exactly 2^k (v_bar included), the other columns are unchanged
+    Q, K, V = _inputs(700, 32, 12)
+    a, _ = oracle.forward_head_mx(Q, K, V, 0.8, 128, pv="e4m3_channel")
+    V2 = V.copy()
+    V2[:, 3] *= 8.0
+    b, _ = oracle.forward_head_mx(Q, K, V2, 0.8, 128, pv="e4m3_channel")
+    assert np.array_equal(b[:, 3], 8.0 * a[:, 3])
+    assert np.array_equal(np.delete(b, 3, axis=1), np.delete(a, 3, axis=1))
+
+
+def test_e4m3_channel_reference_lag_moves_only_subnormal_weights():
+    # a reference lower by k in [1, 4] (an online kernel's integer running maximum with a lazy
+    # threshold of 4) scales every weight by 2^k: P <= 2^(4 + k) <= 256 < 448, so normal weights
+    # scale exactly and only those below 2^-6 round differently; O moves by far less than the
+    # format's own error (one half step of E4M3 is 2^-4 relative)
+    Q, K, V = _inputs(700, 64, 13)
+    base, _ = oracle.forward_head_mx(Q, K, V, 0.8, 128, 1, pv="e4m3_channel")
+    for shift in (-1, -2, -4):
+        O, _ = oracle.forward_head_mx(Q, K, V, 0.8, 128, 1, pv="e4m3_channel", m_shift=shift)
+        assert np.max(np.abs(O - base)) <= 5e-3 and np.abs(O - base).mean() <= 2e-4
+    # past the budget (headroom 4 + lag 6 > 8 binades) the largest weights saturate at 448
+    O, _ = oracle.forward_head_mx(Q, K, V, 0.8, 128, 1, pv="e4m3_channel", m_shift=-6)
+    assert np.max(np.abs(O - base)) > 5e-3
+
+
+def test_e4m3_channel_error_against_the_exact_definition_on_a_seeded_case():
+    # a regression record of this reading's accuracy on one seeded case (int8 scores)
+    Q, K, V = _inputs(1000, 128, 10)
+    ref, _, _, _ = oracle.forward_head(Q, K, V, 0.8, 128, 128, 0)
+    e = np.abs(oracle.forward_head_mx(Q, K, V, 0.8, 128, pv="e4m3_channel")[0] - ref)
+    assert e.mean() < 0.03 and e.max() < 0.5
+
+
 # ---- planted mistakes: each must make at least one pin above fail ------------------------------
 
 def _run_lowp_pins():
@@ -198,6 +283,10 @@ def _run_lowp_pins():
         "routing": lambda: test_routing_is_the_bf16_routing("int8"),
         "exact": lambda: test_exact_operands_reproduce_the_bf16_definition(700, 64, 0.8, 1, True),
         "exact_tau0": lambda: test_exact_operands_reproduce_the_bf16_definition(700, 64, 0.0, 0, True),
+        "channel_scales": test_channel_scales_hand_example,
+        "channel_quantize": test_e4m3_channel_quantize_hand_example,
+        "channel_closed_form": test_e4m3_channel_reading_is_exact_on_a_closed_form_case,
+        "channel_columns": test_e4m3_channel_values_take_the_channel_scale_and_pooled_values_take_v_scales,
     }
     failed = []
     for name, fn in checks.items():
@@ -254,3 +343,37 @@ def test_planted_int8_scale_is_caught(monkeypatch):
     monkeypatch.setattr(mx, "int8_quantize_tiles", wrong)
     monkeypatch.setattr(oracle, "int8_quantize_tiles", wrong)
     assert "int8" in _run_lowp_pins()
+
+
+def test_planted_int8_style_channel_scale_is_caught(monkeypatch):
+    def wrong(V):
+        amax = np.abs(np.asarray(V, dtype=np.float64)).max(axis=0)
+        return np.where(amax > 0, amax / 127.0, 1.0)
+
+    monkeypatch.setattr(mx, "channel_scales", wrong)
+    monkeypatch.setattr(oracle, "channel_scales", wrong)
+    assert "channel_scales" in _run_lowp_pins()
+
+
+def test_planted_per_tensor_channel_scale_is_caught(monkeypatch):
+    def per_tensor(V):
+        a = float(np.abs(np.asarray(V, dtype=np.float64)).max())
+        return np.full(np.shape(V)[1], a / 448.0 if a > 0 else 1.0)
+
+    monkeypatch.setattr(mx, "channel_scales", per_tensor)
+    monkeypatch.setattr(oracle, "channel_scales", per_tensor)
+    assert "channel_scales" in _run_lowp_pins()
+
+
+def test_planted_reference_without_multiplicity_is_caught(monkeypatch):
+    # the weights' reference must count log2(n_j): without it pooled weights (n_j = 128) exceed 448
+    # under a lagging reference and saturate
+    orig = mx.unit_forward_mx
+
+    def no_weights(*a, **kw):
+        kw["ref_with_weights"] = False
+        return orig(*a, **kw)
+
+    monkeypatch.setattr(mx, "unit_forward_mx", no_weights)
+    with pytest.raises(AssertionError):
+        test_e4m3_channel_reference_lag_moves_only_subnormal_weights()
