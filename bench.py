@@ -424,10 +424,11 @@ def cta_spans(launch, dev, torch, sa):
             "tail_frac": float((end.max() - end.mean()) / span), "busy_frac": float(((end - start) / span).mean())}
 
 
-def measure_int8_qk(w, Q, K, V, kbar, vlp, tau, O_bf16, ws, stream, flops, bf16_fwd_ms, pk, max_over_ranks, barrier,
-                    world):
-    """The 8-bit QK^T variant on the workload at the timed density: CUDA-event time of the
-    quantization pass and of the forward, kept-tile TFLOP/s of the forward (the same FLOP count
+def measure_int8_qk(w, Q, K, V, kbar, vbar, vlp, tau, O_bf16, ws, stream, flops, bf16_fwd_ms, pk, max_over_ranks,
+                    barrier, world):
+    """The 8-bit variants on the workload at the timed density: int8 QK^T with bf16 PV, and int8
+    QK^T with E4M3 PV (the whole kept tile in 8 bits). For each: CUDA-event time of the
+    quantization passes and of the forward, kept-tile TFLOP/s of the forward (the same FLOP count
     as the bf16 line), its ratio to the bf16 forward, and its output's distance from the bf16
     output (the variant's own quantization error)."""
     import torch
@@ -465,7 +466,30 @@ def measure_int8_qk(w, Q, K, V, kbar, vlp, tau, O_bf16, ws, stream, flops, bf16_
            "speedup_vs_bf16_fwd": bf16_fwd_ms / f_ms,
            "vs_bf16_output": {"max_abs": float(diff.max()), "mean_abs": float(diff.mean())},
            "note": "QK^T on int8 tensor cores (kind::i8), PV in bf16; FLOPs counted as for the bf16 line"}
-    del q8, k8, kb8, O8, diff
+    del diff
+    # the whole kept tile in 8 bits: E4M3 weights and values with per-channel scales
+    v8t, vb8t, vsc = sa.sol_attn_quantize_v8(V, vbar, stream=stream)
+
+    def quant_v():
+        sa.sol_attn_quantize_v8(V, vbar, stream=stream)
+
+    def fwd8():
+        sa.sol_attn_fwd_8bit(Q, q8, k8, kb8, qs, ks, kbs, v8t, vb8t, vsc, kbar, tau, w.n_force, O=O8, workspace=ws,
+                             stream=stream)
+
+    qv_ms = timed(quant_v)
+    f8_ms = timed(fwd8)
+    sa.sol_attn_check_device_error(ws)
+    diff = (O8.float() - O_bf16.float()).abs()
+    tflops8 = flops / (f8_ms * 1e-3) / 1e12
+    out["e4m3_pv"] = {
+        "kernel": "sol_fwd_tc_kernel<128, int8 QK^T, E4M3 PV>", "quantize_ms": q_ms + qv_ms, "fwd_ms": f8_ms,
+        "fwd_tflops": world * tflops8, "frac_of_bf16_peak": tflops8 / pk["bf16_tflops"],
+        "speedup_vs_bf16_fwd": bf16_fwd_ms / f8_ms,
+        "vs_bf16_output": {"max_abs": float(diff.max()), "mean_abs": float(diff.mean())},
+        "note": "QK^T on kind::i8, PV on kind::f8f6f4 (E4M3 weights, E4M3 values with one scale per channel); "
+                "FLOPs counted as for the bf16 line"}
+    del q8, k8, kb8, O8, diff, v8t, vb8t, vsc
     return out
 
 
@@ -693,7 +717,7 @@ def run_ours(args, w):
         if w.d == 128:
             step(tau)  # the sweep left another density's output in O
             torch.cuda.synchronize()
-            next_rows["int8_qk"] = measure_int8_qk(w, Q, K, V, kbar, vlp, tau, O, ws, stream, flops, fwd_ms, pk,
+            next_rows["int8_qk"] = measure_int8_qk(w, Q, K, V, kbar, vbar, vlp, tau, O, ws, stream, flops, fwd_ms, pk,
                                                    max_over_ranks, barrier, world)
 
     # end to end through the public API: pinned host inputs in, host output back, every step. The

@@ -6,6 +6,8 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 namespace sol {
@@ -188,6 +190,18 @@ __device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem], kind::f8f6f4 (8-bit float inputs, fp32 accumulate); A is M x K
+// in tensor memory, four 8-bit values per 32-bit column.
+__device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand (sm_100 format: version 1).
 // lbo/sbo are byte offsets: K-major uses sbo = 1024 (8 rows of 128 B) and ignores lbo; MN-major
 // uses lbo = distance between 64-element MN groups and sbo = distance between 8-row K groups.
@@ -220,6 +234,15 @@ __host__ __device__ constexpr uint32_t idesc_s8_s32(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
+// Instruction descriptor, kind::f8f6f4 with E4M3 A/B (format code 0) and fp32 D; A and B K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4)                                   // D format: f32
+         | (0u << 7)                                 // A format: E4M3
+         | (0u << 10)                                // B format: E4M3
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
 // An int32 accumulator value as fp32, exactly for |i| < 2^22: the integer is added to the bit
 // pattern of 1.5 * 2^23, whose float spacing is 1, and 1.5 * 2^23 is subtracted back.
 __device__ __forceinline__ float s32_to_f32_small(uint32_t raw) {
@@ -240,6 +263,20 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^k for an integer-valued k <= 0 (a difference of integer references), built exactly from the
+// exponent field; 0 for k < -126 (and for k = -inf).
+__device__ __forceinline__ float exp2_int(float k) {
+  if (!(k >= -126.f)) return 0.f;
+  return __int_as_float((127 + static_cast<int>(k)) << 23);
+}
+
+// Two E4M3 codes (the low byte is the first) as their exact fp32 values: every E4M3 value is an
+// fp16 value, so the conversion through fp16 is exact.
+__device__ __forceinline__ float2 e4m3x2_to_float2(__nv_fp8x2_storage_t v) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(v, __NV_E4M3);
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
 
 // max(a, b, c) in one instruction (sm_100 three-input max).

@@ -67,6 +67,11 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;    // S buffer b at kColS + 128 b
 constexpr uint32_t kColO = 256;  // O_g at kColO + D g
 constexpr float kRescaleThreshold = 8.0f;  // lazy rescale: only when the row max grows by > 2^8
+// 8-bit PV: P is E4M3 with no scale, against an integer reference 6 below the running max; the
+// lazy threshold drops to 2 so that P stays below 2^(6 + 2) = 256 < 448, and every weight above
+// 2^-12 of the running max is a normal E4M3 value (its mantissa rounded, its exponent exact)
+constexpr int kHeadroom8 = 6;
+constexpr float kRescaleThreshold8 = 2.0f;
 constexpr uint32_t kBarSoftmax = 1;       // named barrier of the 256 softmax threads
 
 // cubic minimax fit of 2^f on [0, 1] with p(0) = 1 (relative error <= 8.6e-5)
@@ -78,7 +83,11 @@ constexpr int kPolyEvery = 0;
 
 // QK8: Q, K and the pooled keys arrive as int8 codes (one 128-byte swizzle atom per row at d = 128)
 // and QK^T runs as kind::i8 with int32 accumulation; V, P and the rest stay bf16.
-template <int D, bool QK8>
+// PV8 (with QK8): V and the pooled values arrive as E4M3 codes with one scale per channel, stored
+// transposed ([d][keys], one 128-byte atom of keys per channel row), P is written as E4M3 against
+// an integer running maximum lowered by 6, and PV runs as kind::f8f6f4; the epilogue applies the
+// channel scales.
+template <int D, bool QK8, bool PV8 = false>
 struct TcCfg {
   static constexpr int NCHUNK = D / 64;                 // 128-byte swizzle atoms per bf16 row
   static constexpr int CHUNK_BYTES = kRows * 128;       // 128 rows x 128 B
@@ -89,8 +98,10 @@ struct TcCfg {
   static constexpr int NV = (D == 128) ? 2 : 4;         // V ring depth
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + QK_TILE_BYTES;
+  static constexpr int V_CHUNKS = PV8 ? 1 : NCHUNK;                       // swizzle atoms per V stage row
+  static constexpr int V_TILE_BYTES = V_CHUNKS * CHUNK_BYTES;             // PV8: d rows x 128 key bytes
   static constexpr int OFF_V = OFF_K + NK * QK_TILE_BYTES;
-  static constexpr int OFF_SBAR = OFF_V + NV * TILE_BYTES;                // float[kMaxKeyBlocks]
+  static constexpr int OFF_SBAR = OFF_V + NV * V_TILE_BYTES;              // float[kMaxKeyBlocks]
   static constexpr int OFF_KLIST = OFF_SBAR + kMaxKeyBlocks * 4;          // u16[kMaxKeyBlocks]
   static constexpr int OFF_BITS = OFF_KLIST + kMaxKeyBlocks * 2;          // u32[kMaxKeyBlocks/32]
   static constexpr int OFF_CLIST = OFF_BITS + kMaxKeyBlocks / 8;          // u16[kMaxKeyBlocks/128]
@@ -109,6 +120,7 @@ struct TcCfg {
   static_assert((kSoftmaxThreads / (D / 8)) * D <= kMaxKeyBlocks, "q_bar partial sums fit in the proxy-score buffer");
   static_assert(kColO + 2 * D <= kTmemCols, "TMEM budget");
   static_assert(!QK8 || D == 128, "8-bit QK^T needs d = 128");
+  static_assert(!PV8 || QK8, "8-bit PV comes with 8-bit QK^T");
 };
 
 struct TcParams {
@@ -127,6 +139,7 @@ struct TcParams {
   const float* q_scale;   // 8-bit QK^T: [BH, nqb] query-tile scales
   const float* k_scale;   // [BH, nkb] key-block scales
   const float* kb_scale;  // [BH, ceil(nkb / 128)] pooled-key chunk scales
+  const float* v_scale;   // 8-bit PV: [BH, D] channel scales of V and v_bar
   unsigned long long* cta_times;  // measurement hook: [2 * cta_capacity] start/finish ns, or null
   int cta_capacity;
   float tau[kMaxHeads];
@@ -160,12 +173,12 @@ __device__ __forceinline__ float max64(const float (&s)[64]) {
   return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
 
-template <int D, bool QK8>
+template <int D, bool QK8, bool PV8>
 __global__ void __launch_bounds__(kThreads, 1)
     sol_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKb,
                       const __grid_constant__ CUtensorMap tmVb, const __grid_constant__ TcParams p) {
-  using C = TcCfg<D, QK8>;
+  using C = TcCfg<D, QK8, PV8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -298,10 +311,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               const bool exact = tp < nk;
               const void* mv = exact ? static_cast<const void*>(&tmV) : static_cast<const void*>(&tmVb);
               const int y = (exact ? static_cast<int>(s_klist[tp]) : static_cast<int>(s_clist[tp - nk])) * kRows;
-              mbar_arrive_expect_tx(bar_vfull + 8 * s, C::TILE_BYTES);
-              for (int c = 0; c < C::NCHUNK; ++c)
-                tma_load_3d(sb + C::OFF_V + s * C::TILE_BYTES + c * C::CHUNK_BYTES, mv, bar_vfull + 8 * s, c * 64,
-                            y, bh);
+              mbar_arrive_expect_tx(bar_vfull + 8 * s, C::V_TILE_BYTES);
+              if constexpr (PV8) {
+                // transposed codes: the box is 128 keys (x, from the tile's first key) x d channel rows
+                tma_load_3d(sb + C::OFF_V + s * C::V_TILE_BYTES, mv, bar_vfull + 8 * s, y, 0, bh);
+              } else {
+                for (int c = 0; c < C::NCHUNK; ++c)
+                  tma_load_3d(sb + C::OFF_V + s * C::V_TILE_BYTES + c * C::CHUNK_BYTES, mv, bar_vfull + 8 * s, c * 64,
+                              y, bh);
+              }
               v_armed[s] = g / C::NV + 1u;
             }
           }
@@ -315,10 +333,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         int w = mbar_wait(bar_list, uphase, s_abort, limit);
         if (w == WAIT_OK) {
           const int T = s_misc[MISC_NK] + s_misc[MISC_NC];
-          constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+          constexpr uint32_t idesc_pv = PV8 ? idesc_e4m3_f32(128, D) : idesc_bf16_f32(128, D, true);
           // base descriptor; a K-step or stage offset is added to the start-address field
-          // (addresses stay below 256 KB, so the 14-bit field never carries)
-          const uint64_t vdesc0 = smem_desc_sw128(sb + C::OFF_V, C::CHUNK_BYTES, 1024) + ((4 * grp * 2048) >> 4);
+          // (addresses stay below 256 KB, so the 14-bit field never carries). bf16: V rows
+          // [64 grp, 64 grp + 64) start 4 grp x 2048 B in; E4M3 (K-major, 128 keys per row): keys
+          // [64 grp, ...) start 64 grp B into every row
+          const uint64_t vdesc0 = PV8 ? smem_desc_sw128(sb + C::OFF_V, 16, 1024) + ((64 * grp) >> 4)
+                                      : smem_desc_sw128(sb + C::OFF_V, C::CHUNK_BYTES, 1024) + ((4 * grp * 2048) >> 4);
           const uint32_t o_acc = tmem + kColO + D * grp;
           for (int t = 0; t < T && w == WAIT_OK; ++t) {
             const uint32_t g = tile_base + t;
@@ -328,11 +349,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (w == WAIT_OK) w = mbar_wait(bar_vfull + 8 * s, (g / C::NV) & 1u, s_abort, limit);
             if (w != WAIT_OK) break;
             tc_fence_after();
-            const uint64_t vd = vdesc0 + ((s * C::TILE_BYTES) >> 4);
+            const uint64_t vd = vdesc0 + ((s * C::V_TILE_BYTES) >> 4);
             const uint32_t p_col = tmem + kColS + 128 * b + 64 * grp;
+            if constexpr (PV8) {
+              // 64 keys in two K = 32 steps; P: 32 E4M3 per lane = 8 TMEM columns per step
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ts(o_acc, p_col + kk * 8, vd + ((kk * 2048) >> 4), idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < 2; ++kk)
+                mma_f8_ts(o_acc, p_col + kk * 8, vd + kk * 2, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+            } else {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ts(o_acc, p_col + kk * 8, vd + ((kk * 2048) >> 4), idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+            }
             mma_issued = true;
             tc_commit(bar_vempty + 8 * s);
             tc_commit(bar_pvdone + 8 * b);
@@ -632,45 +660,80 @@ __global__ void __launch_bounds__(kThreads, 1)
         // P = 0, and the first finite max rescales its (zero) accumulator by 0
         float m_new = m_run, alpha = 1.f;
         bool need = false;
-        if (t == 0) {
-          m_new = mx;
-        } else if (mx > m_run + kRescaleThreshold) {
-          need = true;
-          m_new = mx;
-          alpha = ex2_approx(m_run - mx);
-        }
-        m_run = m_new;
-        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-        uint32_t pk[32];
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};  // row sum of the bf16-rounded weights, 4 chains
-        if (full) {
-          const float2 scale2 = make_float2(ts, ts);
-          const float2 negm2 = make_float2(-m_use, -m_use);
-#pragma unroll
-          for (int c2 = 0; c2 < 32; ++c2) {
-            const float2 x2 = __ffma2_rn(make_float2(s[2 * c2], s[2 * c2 + 1]), scale2, negm2);
-            float2 e2;
-            if (kPolyEvery > 0 && (c2 % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
-              e2 = exp2_poly2(make_float2(fmaxf(x2.x, -126.f), fmaxf(x2.y, -126.f)));
-            } else {
-              e2 = make_float2(ex2_approx(x2.x), ex2_approx(x2.y));
-            }
-            pk[c2] = pack_bf16x2(e2.x, e2.y);
-            acc[c2 & 3] = add_bf16x2(acc[c2 & 3], pk[c2]);
+        if constexpr (PV8) {
+          // integer reference (the oracle's e4m3_channel reading): a rescale moves it to the
+          // ceiling of the new max and multiplies O by an exact power of two
+          if (t == 0) {
+            m_new = ceilf(mx);
+          } else if (mx > m_run + kRescaleThreshold8) {
+            need = true;
+            m_new = ceilf(mx);
+            alpha = exp2_int(m_run - m_new);
           }
         } else {
-#pragma unroll
-          for (int c2 = 0; c2 < 32; ++c2) {
-            const float e0 = ex2_approx(s[2 * c2] - m_use);
-            const float e1 = ex2_approx(s[2 * c2 + 1] - m_use);
-            pk[c2] = pack_bf16x2(e0, e1);
-            acc[c2 & 3] = add_bf16x2(acc[c2 & 3], pk[c2]);
+          if (t == 0) {
+            m_new = mx;
+          } else if (mx > m_run + kRescaleThreshold) {
+            need = true;
+            m_new = mx;
+            alpha = ex2_approx(m_run - mx);
           }
         }
-        // the row sum takes the same bf16-rounded weights the PV MMA uses
-        l_run = fmaf(l_run, alpha, (acc[0] + acc[1]) + (acc[2] + acc[3]));
-        // P over the first 32 of this group's S columns, which are already in registers
-        tmem_st_x32(s_col, pk);
+        m_run = m_new;
+        if constexpr (PV8) {
+          // P = 2^(x - (m - 6)) <= 2^(6 + 2) = 256 < 448: E4M3 codes, four per TMEM column; the row
+          // sum adds the codes' exact values, the weights the PV product uses
+          const float m_use = (m_new == -INFINITY) ? 0.f : m_new - static_cast<float>(kHeadroom8);
+          uint32_t pk[16];
+          float2 a2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+          for (int c4 = 0; c4 < 16; ++c4) {
+            float e[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              e[k] = ex2_approx(full ? fmaf(s[4 * c4 + k], ts, -m_use) : s[4 * c4 + k] - m_use);
+            const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(e[0], e[1]), __NV_SATFINITE, __NV_E4M3);
+            const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(e[2], e[3]), __NV_SATFINITE, __NV_E4M3);
+            pk[c4] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+            a2[0] = __fadd2_rn(a2[0], e4m3x2_to_float2(lo));
+            a2[1] = __fadd2_rn(a2[1], e4m3x2_to_float2(hi));
+          }
+          l_run = fmaf(l_run, alpha, (a2[0].x + a2[0].y) + (a2[1].x + a2[1].y));
+          // P over the first 16 of this group's S columns, which are already in registers
+          tmem_st_x16(s_col, pk);
+        } else {
+          const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+          uint32_t pk[32];
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};  // row sum of the bf16-rounded weights, 4 chains
+          if (full) {
+            const float2 scale2 = make_float2(ts, ts);
+            const float2 negm2 = make_float2(-m_use, -m_use);
+#pragma unroll
+            for (int c2 = 0; c2 < 32; ++c2) {
+              const float2 x2 = __ffma2_rn(make_float2(s[2 * c2], s[2 * c2 + 1]), scale2, negm2);
+              float2 e2;
+              if (kPolyEvery > 0 && (c2 % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
+                e2 = exp2_poly2(make_float2(fmaxf(x2.x, -126.f), fmaxf(x2.y, -126.f)));
+              } else {
+                e2 = make_float2(ex2_approx(x2.x), ex2_approx(x2.y));
+              }
+              pk[c2] = pack_bf16x2(e2.x, e2.y);
+              acc[c2 & 3] = add_bf16x2(acc[c2 & 3], pk[c2]);
+            }
+          } else {
+#pragma unroll
+            for (int c2 = 0; c2 < 32; ++c2) {
+              const float e0 = ex2_approx(s[2 * c2] - m_use);
+              const float e1 = ex2_approx(s[2 * c2 + 1] - m_use);
+              pk[c2] = pack_bf16x2(e0, e1);
+              acc[c2 & 3] = add_bf16x2(acc[c2 & 3], pk[c2]);
+            }
+          }
+          // the row sum takes the same bf16-rounded weights the PV MMA uses
+          l_run = fmaf(l_run, alpha, (acc[0] + acc[1]) + (acc[2] + acc[3]));
+          // P over the first 32 of this group's S columns, which are already in registers
+          tmem_st_x32(s_col, pk);
+        }
         if (__any_sync(0xffffffffu, need)) {
           // rescale O_grp once the previous tile's PV has landed. pv_done[buf] completes once per
           // tile using that buffer; the PV three tiles back completed before the one two tiles back
@@ -715,7 +778,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const float2 ml0 = s_ml[row], ml1 = s_ml[kRows + row];
           const float m = fmaxf(ml0.x, ml1.x);  // finite: every row sees at least one valid column
-          const float a0 = ex2_approx(ml0.x - m), a1 = ex2_approx(ml1.x - m);  // 2^-inf = 0
+          // 2^-inf = 0; with integer references (8-bit PV) the factors are exact powers of two
+          const float a0 = PV8 ? exp2_int(ml0.x - m) : ex2_approx(ml0.x - m);
+          const float a1 = PV8 ? exp2_int(ml1.x - m) : ex2_approx(ml1.x - m);
           const float inv = 1.f / fmaf(ml0.y, a0, ml1.y * a1);
           const float c0 = a0 * inv, c1 = a1 * inv;
           const bool store = row < m_i;
@@ -728,10 +793,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld_x32(o0 + ch * 32, x0);
             tmem_ld_x32(o0 + D + ch * 32, x1);
             uint32_t pkd[16];
+            if constexpr (PV8) {
+              // the E4M3 values' channel scales, one per output column
+              const float* vs = p.v_scale + static_cast<size_t>(bh) * D + grp * (D / 2) + ch * 32;
 #pragma unroll
-            for (int c = 0; c < 16; ++c)
-              pkd[c] = pack_bf16x2(fmaf(__uint_as_float(x0[2 * c]), c0, __uint_as_float(x1[2 * c]) * c1),
-                                   fmaf(__uint_as_float(x0[2 * c + 1]), c0, __uint_as_float(x1[2 * c + 1]) * c1));
+              for (int c = 0; c < 16; ++c) {
+                const float2 sc = __ldg(reinterpret_cast<const float2*>(vs) + c);
+                pkd[c] = pack_bf16x2(fmaf(__uint_as_float(x0[2 * c]), c0, __uint_as_float(x1[2 * c]) * c1) * sc.x,
+                                     fmaf(__uint_as_float(x0[2 * c + 1]), c0, __uint_as_float(x1[2 * c + 1]) * c1) *
+                                         sc.y);
+              }
+            } else {
+#pragma unroll
+              for (int c = 0; c < 16; ++c)
+                pkd[c] = pack_bf16x2(fmaf(__uint_as_float(x0[2 * c]), c0, __uint_as_float(x1[2 * c]) * c1),
+                                     fmaf(__uint_as_float(x0[2 * c + 1]), c0, __uint_as_float(x1[2 * c + 1]) * c1));
+            }
             if (store) {
               uint4* d4 = reinterpret_cast<uint4*>(dst + ch * 32);
 #pragma unroll
@@ -783,9 +860,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool QK8>
+template <int D, bool QK8, bool PV8 = false>
 cudaError_t launch_tc_t(const FwdArgs& a, const CUtensorMap* maps, cudaStream_t stream) {
-  using C = TcCfg<D, QK8>;
+  using C = TcCfg<D, QK8, PV8>;
   TcParams p;
   p.kbar = a.kbar;
   p.bits = a.route_bits;
@@ -809,14 +886,16 @@ cudaError_t launch_tc_t(const FwdArgs& a, const CUtensorMap* maps, cudaStream_t 
   p.q_scale = QK8 ? a.qk8->q_scale : nullptr;
   p.k_scale = QK8 ? a.qk8->k_scale : nullptr;
   p.kb_scale = QK8 ? a.qk8->kb_scale : nullptr;
+  p.v_scale = PV8 ? a.pv8->v_scale : nullptr;
   p.cta_times = a.cta_times;
   p.cta_capacity = a.cta_capacity;
   for (int h = 0; h < kMaxHeads; ++h) p.tau[h] = h < a.H ? a.tau[h] : 0.f;
-  cudaError_t e = cudaFuncSetAttribute(sol_fwd_tc_kernel<D, QK8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(sol_fwd_tc_kernel<D, QK8, PV8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int grid = p.total_units < a.num_sms ? p.total_units : a.num_sms;
-  sol_fwd_tc_kernel<D, QK8><<<grid, kThreads, C::SMEM_BYTES, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
+  sol_fwd_tc_kernel<D, QK8, PV8><<<grid, kThreads, C::SMEM_BYTES, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
+                                                                             p);
   return cudaGetLastError();
 }
 
@@ -825,10 +904,12 @@ cudaError_t launch_tc_t(const FwdArgs& a, const CUtensorMap* maps, cudaStream_t 
 cudaError_t launch_fwd_tc(const FwdArgs& a, const CUtensorMap* maps, cudaStream_t stream) {
   if (a.qk8 != nullptr) {
     // 8-bit QK^T: d = 128 and keep bits from the routing pass (the Q tile in shared memory holds
-    // int8 codes, which the in-kernel routing cannot average)
+    // int8 codes, which the in-kernel routing cannot average); 8-bit PV only with it
     if (a.d != 128 || a.route_bits == nullptr) return cudaErrorNotSupported;
+    if (a.pv8 != nullptr) return launch_tc_t<128, true, true>(a, maps, stream);
     return launch_tc_t<128, true>(a, maps, stream);
   }
+  if (a.pv8 != nullptr) return cudaErrorNotSupported;
   if (a.d == 64) return launch_tc_t<64, false>(a, maps, stream);
   if (a.d == 128) return launch_tc_t<128, false>(a, maps, stream);
   return cudaErrorInvalidValue;

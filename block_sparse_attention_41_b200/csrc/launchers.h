@@ -18,6 +18,13 @@ struct Qk8Operands {
   const float* kb_scale;   // [BH, ceil(N_kb / 128)]
 };
 
+// 8-bit PV operands of the forward (sol_attn_quantize_v8): E4M3 codes, transposed, and channel scales
+struct Pv8Operands {
+  const uint8_t* v8t;      // [BH, d, N_kb * 128]
+  const uint8_t* vb8t;     // [BH, d, 128 * ceil(N_kb / 128)]
+  const float* v_scale;    // [BH, d]
+};
+
 struct FwdArgs {
   const void* Q;
   const void* K;
@@ -44,6 +51,7 @@ struct FwdArgs {
   unsigned long long* cta_times = nullptr;  // measurement hook: [2 * cta_capacity] start/finish ns
   int cta_capacity = 0;
   const Qk8Operands* qk8 = nullptr;  // bf16 path: int8 Q, K and pooled keys for QK^T, or null
+  const Pv8Operands* pv8 = nullptr;  // with qk8: E4M3 V and v_bar for PV (kind::f8f6f4), or null
   const float* qbar_in = nullptr;    // routing pass: fp32 [B*H, N_qb, d] query-block means given by the
                                      // caller (the QK-norm + RoPE pass); null = computed from Q
 };
@@ -87,6 +95,17 @@ struct QuantArgs {
 // bf16, d in {64, 128}, blocks of 128: the mean key, then int8 codes and tile scales of Q, K - mu
 // and k_bar - mu.
 cudaError_t launch_quant_qk8(const QuantArgs& a, cudaStream_t stream);
+
+// 8-bit PV values (d = 128): per-channel scales of V and the transposed E4M3 codes of V and v_bar.
+struct QuantV8Args {
+  const void* V;        // bf16 [BH, L, d]
+  const float* vbar;    // fp32 [BH, N_kb, d] from the pooling pass
+  uint8_t* v8t;         // out: E4M3 [BH, d, N_kb * 128], keys contiguous, zero past L
+  uint8_t* vb8t;        // out: E4M3 [BH, d, 128 * ceil(N_kb / 128)], zero past N_kb
+  float* v_scale;       // out: fp32 [BH, d] (also the amax accumulator while the pass runs)
+  int BH, L, d;
+};
+cudaError_t launch_quant_v8(const QuantV8Args& a, cudaStream_t stream);
 
 // bf16, d in {64, 128}: QK RMS norm + rotary embedding + K/V block pooling in one pass.
 cudaError_t launch_qknorm_rope_pool(const RopePoolArgs& a, cudaStream_t stream);

@@ -15,6 +15,7 @@
 // row, keeps the tile's values in registers between the amax pass and the code pass, and writes
 // 8 (bf16 input) or 4 (fp32 input) codes at a time.
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 
 #include "device_common.cuh"
 #include "launchers.h"
@@ -156,12 +157,117 @@ cudaError_t launch_quant_d(const QuantArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// ---- 8-bit PV values: V and v_bar as E4M3 with one scale per channel (d = 128) -----------------
+// SageAttention's FP8 PV layout: s_c = amax_c / 448 over the head's L tokens (1 for an all-zero
+// channel); a code is E4M3(x / s_c), round to nearest even, saturating at +-448. The codes are
+// stored transposed, [d][keys] per head (keys contiguous), the K-major layout of the PV product's
+// B operand; keys past L (and pooled blocks past N_kb) get code 0. v_bar takes V's scales.
+
+constexpr int kVD = 128;
+
+// Per-(head, channel) amax of V over one 128-key block, merged into amax[] with atomicMax on the
+// float bits (non-negative floats order as their bit patterns).
+__global__ void __launch_bounds__(256) sol_v_amax_kernel(const __nv_bfloat16* __restrict__ V,
+                                                         unsigned int* __restrict__ amax, int L) {
+  __shared__ float s_m[16][kVD];  // [row group][channel]
+  const int j = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
+  const int cg = t & 15, rg = t >> 4;  // channels [8 cg, 8 cg + 8), rows rg, rg + 16, ...
+  const int n = min(kTileRows, L - j * kTileRows);
+  const __nv_bfloat16* base = V + (static_cast<size_t>(bh) * L + static_cast<size_t>(j) * kTileRows) * kVD + cg * 8;
+  float m[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m[k] = 0.f;
+  for (int r = rg; r < n; r += 16) {
+    float x[8];
+    Vec<__nv_bfloat16>::unpack(__ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(r) * kVD)), x);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m[k] = fmaxf(m[k], fabsf(x[k]));
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) s_m[rg][cg * 8 + k] = m[k];
+  __syncthreads();
+  if (t < kVD) {
+    float a = 0.f;
+#pragma unroll
+    for (int g = 0; g < 16; ++g) a = fmaxf(a, s_m[g][t]);
+    atomicMax(amax + static_cast<size_t>(bh) * kVD + t, __float_as_uint(a));
+  }
+}
+
+__device__ __forceinline__ float channel_scale(unsigned int amax_bits) {
+  const float a = __uint_as_float(amax_bits);
+  return a > 0.f ? a / 448.f : 1.f;
+}
+
+// Codes of 128 rows (tokens or pooled blocks) of one head, written transposed: out[c][col0 + r].
+// T = bf16 (V, 8 channels per 16-byte load) or float (v_bar, 4 per load).
+template <typename T>
+__global__ void __launch_bounds__(256) sol_v_codes_kernel(const T* __restrict__ src, const unsigned int* __restrict__ amax,
+                                                          uint8_t* __restrict__ out, int rows, int out_pitch) {
+  constexpr int VEC = Vec<T>::N;
+  constexpr int CG = kVD / VEC;     // channel groups per row
+  constexpr int RG = 256 / CG;      // row groups
+  __shared__ uint8_t s_codes[kVD][kTileRows + 16];  // [channel][row], rows padded to 144 B
+  __shared__ float s_scale[kVD];
+  const int jb = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
+  if (t < kVD) s_scale[t] = channel_scale(__ldg(amax + static_cast<size_t>(bh) * kVD + t));
+  __syncthreads();
+  const int cg = t % CG, rg = t / CG;
+  const int n = min(kTileRows, rows - jb * kTileRows);
+  const T* base = src + (static_cast<size_t>(bh) * rows + static_cast<size_t>(jb) * kTileRows) * kVD + cg * VEC;
+  for (int r = rg; r < kTileRows; r += RG) {
+    float x[VEC];
+    if (r < n) {
+      Vec<T>::unpack(__ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(r) * kVD)), x);
+    } else {
+#pragma unroll
+      for (int k = 0; k < VEC; ++k) x[k] = 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < VEC; ++k) {
+      const int c = cg * VEC + k;
+      s_codes[c][r] = static_cast<uint8_t>(__nv_cvt_float_to_fp8(__fdiv_rn(x[k], s_scale[c]), __NV_SATFINITE, __NV_E4M3));
+    }
+  }
+  __syncthreads();
+  // thread t writes 64 codes (keys or pooled blocks [64 h, 64 h + 64)) of channel t / 2
+  const int c = t >> 1, h = t & 1;
+  uint8_t* dst = out + (static_cast<size_t>(bh) * kVD + c) * out_pitch + static_cast<size_t>(jb) * kTileRows + 64 * h;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    *reinterpret_cast<uint4*>(dst + 16 * i) = *reinterpret_cast<const uint4*>(&s_codes[c][64 * h + 16 * i]);
+}
+
+// amax bits -> scales, in place
+__global__ void __launch_bounds__(kVD) sol_v_scale_kernel(unsigned int* amax_then_scale) {
+  const size_t i = static_cast<size_t>(blockIdx.x) * kVD + threadIdx.x;
+  amax_then_scale[i] = __float_as_uint(channel_scale(amax_then_scale[i]));
+}
+
 }  // namespace
 
 cudaError_t launch_quant_qk8(const QuantArgs& a, cudaStream_t stream) {
   if (a.d == 64) return launch_quant_d<64>(a, stream);
   if (a.d == 128) return launch_quant_d<128>(a, stream);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_quant_v8(const QuantV8Args& a, cudaStream_t stream) {
+  if (a.d != kVD) return cudaErrorInvalidValue;
+  const int nkb = (a.L + kTileRows - 1) / kTileRows;
+  const int nchunks = (nkb + kTileRows - 1) / kTileRows;
+  unsigned int* amax = reinterpret_cast<unsigned int*>(a.v_scale);
+  cudaError_t e = cudaMemsetAsync(amax, 0, static_cast<size_t>(a.BH) * kVD * 4, stream);
+  if (e != cudaSuccess) return e;
+  sol_v_amax_kernel<<<dim3(nkb, a.BH), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.V), amax, a.L);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  sol_v_codes_kernel<__nv_bfloat16><<<dim3(nkb, a.BH), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.V), amax,
+                                                                         a.v8t, a.L, nkb * kTileRows);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  sol_v_codes_kernel<float><<<dim3(nchunks, a.BH), 256, 0, stream>>>(a.vbar, amax, a.vb8t, nkb, nchunks * kTileRows);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  sol_v_scale_kernel<<<a.BH, kVD, 0, stream>>>(amax);
+  return cudaGetLastError();
 }
 
 }  // namespace sol

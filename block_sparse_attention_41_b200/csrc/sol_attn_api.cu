@@ -350,7 +350,8 @@ sol_status fwd_impl(const void* Q, const void* K, const void* V, const float* kb
                     const void* kbar_lp, const void* vbar_lp, const float* tau, sol_dtype dt, int B, int H, int L,
                     int d, int block_q, int block_k, int n_force, void* O, uint8_t* kept_mask, float* density,
                     void* workspace, size_t ws_bytes, void* stream, int k_keep,
-                    const sol::Qk8Operands* qk8 = nullptr, const float* qbar_in = nullptr) {
+                    const sol::Qk8Operands* qk8 = nullptr, const float* qbar_in = nullptr,
+                    const sol::Pv8Operands* pv8 = nullptr) {
   if (dt != SOL_F32 && dt != SOL_BF16) return fail(SOL_EINVAL, "unknown dtype %d", static_cast<int>(dt));
   if (!size_ok(B, 1 << 16) || !size_ok(H, 1 << 16) || !size_ok(L, 1 << 28) || !size_ok(d, 1 << 16) ||
       !size_ok(block_q, 1 << 20) || !size_ok(block_k, 1 << 20))
@@ -442,10 +443,19 @@ sol_status fwd_impl(const void* Q, const void* K, const void* V, const float* kb
     const bool i8 = qk8 != nullptr;  // Q, K and the pooled keys as int8 codes
     if ((st = make_map(&maps[0], i8 ? qk8->q8 : Q, d, L, B * H, i8)) != SOL_OK) return st;
     if ((st = make_map(&maps[1], i8 ? qk8->k8 : K, d, L, B * H, i8)) != SOL_OK) return st;
-    if ((st = make_map(&maps[2], V, d, L, B * H)) != SOL_OK) return st;
+    if (pv8 != nullptr) {
+      // E4M3 codes stored transposed: rows are the d channels, the inner extent runs over keys
+      // (N_kb * 128) or pooled blocks (128 * ceil(N_kb / 128))
+      const int cp = (nkb_i + 127) / 128 * 128;
+      if ((st = make_map(&maps[2], pv8->v8t, nkb_i * 128, d, B * H, true)) != SOL_OK) return st;
+      if ((st = make_map(&maps[4], pv8->vb8t, cp, d, B * H, true)) != SOL_OK) return st;
+    } else {
+      if ((st = make_map(&maps[2], V, d, L, B * H)) != SOL_OK) return st;
+      if ((st = make_map(&maps[4], vbar_lp, d, nkb_i, B * H)) != SOL_OK) return st;
+    }
     if ((st = make_map(&maps[3], i8 ? qk8->kb8 : kbar_lp, d, nkb_i, B * H, i8)) != SOL_OK) return st;
-    if ((st = make_map(&maps[4], vbar_lp, d, nkb_i, B * H)) != SOL_OK) return st;
     a.qk8 = qk8;
+    a.pv8 = pv8;
     a.qbar_in = route_pass ? qbar_in : nullptr;
     if (route_pass) {
       e = sol::launch_route(a, s);
@@ -520,6 +530,60 @@ sol_status sol_attn_fwd_qk8(const void* Q, const int8_t* q8, const int8_t* k8, c
   // K is not read on this path; k8 stands in for it in the argument checks
   return fwd_impl(Q, k8, V, kbar, nullptr, vbar_lp, vbar_lp, tau, SOL_BF16, B, H, L, d, 128, 128, n_force, O,
                   kept_mask, density, workspace, ws_bytes, stream, 0, &ops);
+}
+
+sol_status sol_attn_quantize_v8(const void* V, const float* vbar, int B, int H, int L, int d, uint8_t* v8t,
+                                uint8_t* vbar8t, float* v_scale, void* stream) {
+  g_last_error.clear();
+  if (!size_ok(B, 1 << 16) || !size_ok(H, 1 << 16) || !size_ok(L, 1 << 28) || !size_ok(d, 1 << 16))
+    return fail(SOL_EINVAL, "sizes must be positive (B=%d H=%d L=%d d=%d)", B, H, L, d);
+  const void* ptrs[] = {V, vbar, v8t, vbar8t, v_scale};
+  for (const void* ptr : ptrs) {
+    if (ptr == nullptr) return fail(SOL_EINVAL, "every pointer argument must be non-null");
+    if (!aligned16(ptr)) return fail(SOL_EINVAL, "device pointers must be 16-byte aligned");
+  }
+  if (d != 128) return fail(SOL_EUNSUPPORTED, "8-bit PV values need d = 128 (d=%d)", d);
+  if (static_cast<long long>(B) * H > 65535) return fail(SOL_EUNSUPPORTED, "B*H must be <= 65535");
+  const long long nkb = (static_cast<long long>(L) + 127) / 128;
+  if (nkb > sol::kMaxKeyBlocks) return fail(SOL_EUNSUPPORTED, "N_kb=%lld exceeds %d", nkb, sol::kMaxKeyBlocks);
+  int sms = 0;
+  sol_status st = current_device(&sms);
+  if (st != SOL_OK) return st;
+  sol::QuantV8Args a;
+  a.V = V;
+  a.vbar = vbar;
+  a.v8t = v8t;
+  a.vb8t = vbar8t;
+  a.v_scale = v_scale;
+  a.BH = B * H;
+  a.L = L;
+  a.d = d;
+  cudaError_t e = sol::launch_quant_v8(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "8-bit value quantization launch");
+  return SOL_OK;
+}
+
+sol_status sol_attn_fwd_8bit(const void* Q, const int8_t* q8, const int8_t* k8, const int8_t* kbar8,
+                             const float* q_scale, const float* k_scale, const float* kbar_scale, const uint8_t* v8t,
+                             const uint8_t* vbar8t, const float* v_scale, const float* kbar, const float* tau, int B,
+                             int H, int L, int d, int n_force, void* O, uint8_t* kept_mask, float* density,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  if (B < 1 || H < 1 || L < 1) return fail(SOL_EINVAL, "sizes must be positive (B=%d H=%d L=%d)", B, H, L);
+  const void* ptrs[] = {q8, k8, kbar8, q_scale, k_scale, kbar_scale, v8t, vbar8t, v_scale};
+  for (const void* ptr : ptrs) {
+    if (ptr == nullptr) return fail(SOL_EINVAL, "every 8-bit operand and scale must be non-null");
+    if (!aligned16(ptr)) return fail(SOL_EINVAL, "device pointers must be 16-byte aligned");
+  }
+  if (d != 128) return fail(SOL_EUNSUPPORTED, "8-bit attention needs d = 128 (d=%d)", d);
+  if (workspace == nullptr || ws_bytes < sol_attn_fwd_workspace_bytes(B, H, L, 128))
+    return fail(SOL_EINVAL, "8-bit attention needs the full workspace (its routing pass reads the bf16 Q)");
+  sol::Qk8Operands qk{q8, k8, kbar8, q_scale, k_scale, kbar_scale};
+  sol::Pv8Operands pv{v8t, vbar8t, v_scale};
+  // K, V and the bf16 pooled values are not read on this path; 8-bit operands stand in for them
+  // in the argument checks
+  return fwd_impl(Q, k8, v8t, kbar, nullptr, vbar8t, vbar8t, tau, SOL_BF16, B, H, L, d, 128, 128, n_force, O,
+                  kept_mask, density, workspace, ws_bytes, stream, 0, &qk, nullptr, &pv);
 }
 
 sol_status sol_attn_fwd_noalloc(const void* Q, const void* K, const void* V, const float* kbar, const float* vbar,

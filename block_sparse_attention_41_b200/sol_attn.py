@@ -39,6 +39,8 @@ EXPORTED = (
     "sol_attn_fwd_qk8",
     "sol_attn_qknorm_rope_pool_qbar",
     "sol_attn_fwd_qbar",
+    "sol_attn_quantize_v8",
+    "sol_attn_fwd_8bit",
 )
 
 
@@ -87,6 +89,11 @@ def load_library() -> ctypes.CDLL:
     lib.sol_attn_fwd_qbar.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, f32p, i32, i32, i32, i32, i32, vp, vp, vp, vp,
                                       ctypes.c_size_t, vp]
     lib.sol_attn_fwd_qbar.restype = i32
+    lib.sol_attn_quantize_v8.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp]
+    lib.sol_attn_quantize_v8.restype = i32
+    lib.sol_attn_fwd_8bit.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, f32p, i32, i32, i32, i32, i32, vp, vp,
+                                      vp, vp, ctypes.c_size_t, vp]
+    lib.sol_attn_fwd_8bit.restype = i32
     lib.sol_attn_quantize_qk8.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.sol_attn_quantize_qk8.restype = i32
     lib.sol_attn_fwd_qk8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, f32p, i32, i32, i32, i32, i32, vp, vp,
@@ -378,6 +385,48 @@ def sol_attn_fwd_qbar(Q, K, V, kbar, vbar, kbar_lp, vbar_lp, qbar, tau, n_force:
         _ptr(Q), _ptr(K), _ptr(V), _ptr(kbar), _ptr(vbar), _ptr(kbar_lp), _ptr(vbar_lp), _ptr(qbar), tau_arr, B, H, L,
         d, int(n_force), _ptr(O), _ptr(kept_mask), _ptr(density), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "sol_attn_fwd_qbar")
+    return O
+
+
+def sol_attn_quantize_v8(V, vbar, stream=None):
+    """8-bit PV values (d = 128, blocks of 128): returns (v8t, vbar8t, v_scale), the E4M3 codes of V
+    and of the pooled values vbar with one scale amax_c / 448 per channel, stored transposed
+    ([B, H, d, N_kb * 128] and [B, H, d, 128 * ceil(N_kb / 128)], uint8)."""
+    _need_cuda("V", V, torch.bfloat16)
+    _need_cuda("vbar", vbar, torch.float32)
+    B, H, L, d = V.shape
+    nkb = -(-L // 128)
+    if tuple(vbar.shape) != (B, H, nkb, d):
+        raise ValueError("vbar must be [B, H, ceil(L/128), d]")
+    dev = V.device
+    v8t = torch.empty((B, H, d, nkb * 128), dtype=torch.uint8, device=dev)
+    vbar8t = torch.empty((B, H, d, -(-nkb // 128) * 128), dtype=torch.uint8, device=dev)
+    v_scale = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+    st = load_library().sol_attn_quantize_v8(_ptr(V), _ptr(vbar), B, H, L, d, _ptr(v8t), _ptr(vbar8t),
+                                             _ptr(v_scale), _stream(stream))
+    _check(st, "sol_attn_quantize_v8")
+    return v8t, vbar8t, v_scale
+
+
+def sol_attn_fwd_8bit(Q, q8, k8, kbar8, q_scale, k_scale, kbar_scale, v8t, vbar8t, v_scale, kbar, tau,
+                      n_force: int = 0, O=None, kept_mask=None, density=None, workspace=None, stream=None):
+    """Fused forward with 8-bit kept tiles and correction: int8 QK^T (sol_attn_quantize_qk8) and E4M3
+    PV (sol_attn_quantize_v8); routing from the bf16 Q and the fp32 pooled keys. Returns O (bf16)."""
+    _need_cuda("Q", Q, torch.bfloat16)
+    B, H, L, d = Q.shape
+    tau = [float(x) for x in tau]
+    if len(tau) != H:
+        raise ValueError(f"tau must hold H={H} values")
+    tau_c = (ctypes.c_float * H)(*tau)
+    if O is None:
+        O = torch.empty_like(Q)
+    if workspace is None:
+        workspace = new_workspace(B, H, L, 128, Q.device)
+    st = load_library().sol_attn_fwd_8bit(
+        _ptr(Q), _ptr(q8), _ptr(k8), _ptr(kbar8), _ptr(q_scale), _ptr(k_scale), _ptr(kbar_scale), _ptr(v8t),
+        _ptr(vbar8t), _ptr(v_scale), _ptr(kbar), tau_c, B, H, L, d, int(n_force), _ptr(O), _ptr(kept_mask),
+        _ptr(density), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "sol_attn_fwd_8bit")
     return O
 
 

@@ -137,6 +137,37 @@ sol_status sol_attn_quantize_qk8(const void* Q, const void* K, const float* kbar
                                  int d, int8_t* q8, int8_t* k8, int8_t* kbar8, float* q_scale,
                                  float* k_scale, float* kbar_scale, float* mu, void* stream);
 
+/* 8-bit values for PV (NEXT-2, the "e4m3_channel" reading of SageAttention's FP8 PV: V in E4M3
+ * with one scale per channel). From V (bf16 [B, H, L, d]) and the fp32 pooled values vbar of
+ * sol_attn_pool, with blocks of 128:
+ *   v_scale   device, out, float32 [B, H, d]: amax_c / 448 of each channel over the head's L
+ *             tokens (1 for an all-zero channel)
+ *   v8t       device, out, uint8 (E4M3 codes) [B, H, d, N_kb * 128]: E4M3(V[t, c] / v_scale[c]),
+ *             round to nearest even, saturating; transposed (tokens contiguous), 0 past L
+ *   vbar8t    device, out, uint8 (E4M3 codes) [B, H, d, 128 * ceil(N_kb / 128)]: vbar with the same
+ *             channel scales, transposed, 0 past N_kb
+ * d = 128, N_kb <= 4096, B*H <= 65535, all pointers non-null and 16-byte aligned. Asynchronous on
+ * `stream`; v_scale doubles as the per-channel maximum while the pass runs. */
+sol_status sol_attn_quantize_v8(const void* V, const float* vbar, int B, int H, int L, int d,
+                                uint8_t* v8t, uint8_t* vbar8t, float* v_scale, void* stream);
+
+/* The forward with 8-bit kept tiles and correction (NEXT-2): QK^T from the int8 codes of
+ * sol_attn_quantize_qk8 (kind::i8), PV from E4M3 weights and the E4M3 values of
+ * sol_attn_quantize_v8 (tcgen05 kind::f8f6f4, fp32 accumulation). Each softmax group keeps an
+ * integer running maximum m (a lazy rescale when a tile's max passes m + 2 moves it to the
+ * ceiling of the new max and scales the accumulator by an exact power of two) and writes
+ * P = E4M3(2^(l log2(e) + log2(n_j) - (m - 6))) <= 256, so every weight above 2^-12 of the
+ * running max keeps E4M3's mantissa rounding with an exact exponent; the row sum adds those E4M3
+ * values; the epilogue multiplies output column c by v_scale[c]. Routing is sol_attn_fwd's (bf16 Q, fp32
+ * pooled keys kbar). SOL_BF16 semantics for O, d = 128, blocks of 128, the full workspace of
+ * sol_attn_fwd_workspace_bytes. Other arguments, limits and errors as for sol_attn_fwd. */
+sol_status sol_attn_fwd_8bit(const void* Q, const int8_t* q8, const int8_t* k8, const int8_t* kbar8,
+                             const float* q_scale, const float* k_scale, const float* kbar_scale,
+                             const uint8_t* v8t, const uint8_t* vbar8t, const float* v_scale,
+                             const float* kbar, const float* tau, int B, int H, int L, int d,
+                             int n_force, void* O, uint8_t* kept_mask, float* density, void* workspace,
+                             size_t ws_bytes, void* stream);
+
 /* Bytes of device workspace sol_attn_fwd needs for this problem. The workspace holds the
  * persistent scheduler's work counter, the per-(b,h) kept-block counters and the sticky device
  * error word (a header of 4 * (4 + B*H) bytes rounded up to 256), followed by the routing pass's

@@ -28,6 +28,7 @@ from .mxfp8_oracle import (  # noqa: F401
     mx_quantize,
     no_quantize,
     round_e4m3,
+    round_mantissa,
 )
 from .topk_routing_oracle import forward_head_topk, keep_count, route_topk  # noqa: F401
 from .taylor_correction_oracle import cross_moments, forward_head_taylor, unit_forward_taylor  # noqa: F401

@@ -35,16 +35,14 @@ the plainest reading that a Blackwell block-scaled tensor-core kernel computes:
   O_r = sum_tiles Pq_tile Vq_tile / sum_tiles sum(Pq_tile).
 
 A second PV reading, "e4m3_channel" (SageAttention's own PV layout, where V is FP8 with one scale
-per channel): P is E4M3 with no block scale, and V is E4M3 with one scale per channel,
-s_c = amax_c / 448 over all of the head's tokens. The pooled values v_bar use the same channel scales
-(their entries lie within each channel's range). Without a block scale the weights need a
-reference that bounds them: here M_r is the ceiling of the row's largest l log2(e) + log2(w) (the
-multiplicity counted, as an online kernel's running maximum counts it), lowered by P_HEADROOM = 4,
-so P <= 2^4 and the weights keep 4 more binades above E4M3's subnormals. An online kernel whose
-integer running maximum lags M_r by k in [0, 4] (a lazy rescale threshold of 4) holds
-2^k P <= 256 < 448: every normal E4M3 weight scales exactly, and only weights below 2^-6 (E4M3's
-subnormals, step 2^-9) round differently. A channel scale is one factor on an output column:
-O_rc = s_c sum_t Pq_rt Vcode_tc / sum_t Pq_rt.
+per channel): V is E4M3 with one scale per channel, s_c = amax_c / 448 over all of the head's
+tokens, and the pooled values v_bar use the same channel scales (their entries lie within each
+channel's range). P carries no block scale: each weight keeps E4M3's 3 stored mantissa bits (round
+to nearest even), with its exponent left to the kernel. An online kernel keeps P's exponent inside
+E4M3's normal range relative to its own integer running maximum, so this rounding is the one it
+applies to every weight that matters; and it commutes with any power-of-two reference, so the
+result does not depend on the reference or the order of the tiles. A channel scale is one factor
+on an output column: O_rc = s_c sum_t Pq_rt Vcode_tc / sum_t Pq_rt.
 
 Parity with an upstream low-precision kernel is unpinned: the pages give no formula. The pins
 in tests/test_oracle_lowp_pins.py tie this oracle to the OCP formats' definitions and to the bf16
@@ -66,7 +64,6 @@ E4M3_EMIN = -6     # smallest normal exponent; subnormals are multiples of 2^-9
 E4M3_MANT = 3      # stored mantissa bits
 MX_BLOCK = 32      # values sharing one scale
 TILE = 128         # columns of one P tile (one key block, or one chunk of pooled blocks)
-P_HEADROOM = 4     # "e4m3_channel": binades between the largest weight and the reference
 
 
 def round_e4m3(x):
@@ -122,10 +119,18 @@ def e4m3_channel_quantize(x, scales):
     return round_e4m3(np.asarray(x, dtype=np.float64) / s) * s
 
 
+def round_mantissa(x, bits=E4M3_MANT):
+    """x with its significand rounded to 1 + `bits` bits (round to nearest, ties to even) and an
+    unbounded exponent: no underflow, no saturation."""
+    x = np.asarray(x, dtype=np.float64)
+    f, e = np.frexp(x)                                   # x = f 2^e, |f| in [0.5, 1)
+    return np.ldexp(np.round(np.ldexp(f, bits + 1)), e - bits - 1)
+
+
 def e4m3_plain(x, axis=-1):
-    """E4M3 rounding with no scale: the P of the "e4m3_channel" reading (axis is unused; the
-    signature matches mx_quantize)."""
-    return round_e4m3(x)
+    """The P of the "e4m3_channel" reading: E4M3's mantissa rounding with the exponent left to the
+    kernel (axis is unused; the signature matches mx_quantize)."""
+    return round_mantissa(x)
 
 
 def no_quantize(x, axis=-1):
@@ -133,7 +138,7 @@ def no_quantize(x, axis=-1):
     return np.asarray(x, dtype=np.float64)
 
 
-def unit_forward_mx(qq, Kq, Vq, kbq, vbq, block, n, keep, quant, m_shift=0, ref_with_weights=False):
+def unit_forward_mx(qq, Kq, Vq, kbq, vbq, block, n, keep, quant, m_shift=0):
     """Output rows [m, d] of one query block from its quantized rows qq [m, d], the quantized keys
     and values Kq, Vq [L, d] and pooled ones kbq, vbq [N_kb, d], the valid counts n [N_kb] and
     the routing decision keep [N_kb] (see the module docstring)."""
@@ -162,12 +167,8 @@ def unit_forward_mx(qq, Kq, Vq, kbq, vbq, block, n, keep, quant, m_shift=0, ref_
         w[: cols.size] = np.where(skipped[cols], n[cols].astype(np.float64), 0.0)
         vals[: cols.size] = vbq[cols]  # the whole chunk of pooled values, kept blocks' rows included
         tiles.append((x2, w, vals))
-    # integer reference per row: the ceiling of the largest logit * log2(e) over the used columns,
-    # plus log2 of the column's multiplicity when ref_with_weights
-    def lead(x2, w):
-        lw = np.log2(np.where(w > 0, w, 1.0)) if ref_with_weights else np.zeros_like(w)
-        return np.max(np.where(w[None, :] > 0, x2 + lw[None, :], -np.inf), axis=1)
-    top = np.max([lead(x2, w) for x2, w, _ in tiles], axis=0)
+    # integer reference per row: the ceiling of the largest logit * log2(e) over the used columns
+    top = np.max([np.max(np.where(w[None, :] > 0, x2, -np.inf), axis=1) for x2, w, _ in tiles], axis=0)
     M = np.ceil(top)[:, None] + m_shift
     num = np.zeros((m, d))
     den = np.zeros((m, 1))
@@ -222,7 +223,5 @@ def forward_head_mx(Q, K, V, tau, block, n_force=0, smooth_k=True, quant=mx_quan
         qbar = Q[r0:r1].sum(axis=0) / nq[i]
         keep, _ = route(proxy_scores(qbar, kbar, d), tau, n_force)
         keep_all[i] = keep
-        channel = pv == "e4m3_channel"
-        O[r0:r1] = unit_forward_mx(Qq[r0:r1], Kq, Vq, kbq, vbq, block, n, keep, pq,
-                                   m_shift - (P_HEADROOM if channel else 0), ref_with_weights=channel)
+        O[r0:r1] = unit_forward_mx(Qq[r0:r1], Kq, Vq, kbq, vbq, block, n, keep, pq, m_shift)
     return O, keep_all

@@ -222,3 +222,27 @@ def test_qbar_entries_reject_invalid_arguments(lib):
                                                   1000, 128, 128, P[7], P[8], P[9], P[10], P[11], P[11], qbar, None)
     assert pool(qbar=None) == sa.SOL_EINVAL
     assert "qbar" in lib.sol_attn_last_error().decode()
+
+
+def test_8bit_value_and_forward_entries_reject_invalid_arguments(lib):
+    def quant(d=128, L=1000, ptrs=None):
+        p = list(ptrs or P)
+        return lib.sol_attn_quantize_v8(p[0], p[1], 1, 2, L, d, p[2], p[3], p[4], None)
+    assert quant(d=64) == sa.SOL_EUNSUPPORTED
+    assert quant(L=0) == sa.SOL_EINVAL
+    nulls = list(P)
+    nulls[3] = None
+    assert quant(ptrs=nulls) == sa.SOL_EINVAL
+    assert quant(L=4097 * 128) == sa.SOL_EUNSUPPORTED
+    tau = (ctypes.c_float * 2)(0.5, 0.5)
+
+    def fwd(d=128, ws=1 << 30, ptrs=None):
+        p = list(ptrs or P)
+        return lib.sol_attn_fwd_8bit(p[0], p[1], p[2], p[3], p[4], p[5], p[6], p[7], p[8], p[9], p[10], tau, 1, 2,
+                                     1000, d, 0, p[11], None, None, p[11], ws, None)
+    assert fwd(d=64) == sa.SOL_EUNSUPPORTED
+    assert fwd(ws=256) == sa.SOL_EINVAL
+    assert "full workspace" in lib.sol_attn_last_error().decode()
+    nulls = list(P)
+    nulls[8] = None  # vbar8t
+    assert fwd(ptrs=nulls) == sa.SOL_EINVAL
