@@ -249,16 +249,6 @@ __device__ __forceinline__ float s32_to_f32_small(uint32_t raw) {
   return __int_as_float(static_cast<int>(raw) + 0x4B400000) - 12582912.0f;
 }
 
-// Per-warpgroup register re-balancing (all warps of a warpgroup execute the same one).
-template <uint32_t N>
-__device__ __forceinline__ void regs_increase() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <uint32_t N>
-__device__ __forceinline__ void regs_decrease() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
