@@ -345,8 +345,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t g = tile_base + t;
             const uint32_t b = g & 1u;
             const int s = static_cast<int>(g % C::NV);
-            w = mbar_wait(bar_pfull + 8 * (2 * b + grp), (g >> 1) & 1u, s_abort, limit);
-            if (w == WAIT_OK) w = mbar_wait(bar_vfull + 8 * s, (g / C::NV) & 1u, s_abort, limit);
+            // V first: it lands long before P, so the wait on P is the one left on the critical path
+            w = mbar_wait(bar_vfull + 8 * s, (g / C::NV) & 1u, s_abort, limit);
+            if (w == WAIT_OK) w = mbar_wait(bar_pfull + 8 * (2 * b + grp), (g >> 1) & 1u, s_abort, limit);
             if (w != WAIT_OK) break;
             tc_fence_after();
             const uint64_t vd = vdesc0 + ((s * C::V_TILE_BYTES) >> 4);
@@ -386,8 +387,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             // S[b] holds the P of tile t-2 until that tile's PV has completed. pv_done[b] completes
             // once per tile using S[b], and the PV of tile t cannot run before this QK^T, so the
             // parity wait is exact. (Tiles of the previous unit completed before the unit ended.)
-            if (t >= 2) w = mbar_wait(bar_pvdone + 8 * b, ((g - 2u) >> 1) & 1u, s_abort, limit);
-            if (w == WAIT_OK) w = mbar_wait(bar_kfull + 8 * s, (g / C::NK) & 1u, s_abort, limit);
+            // K first (loaded well ahead), then the PV that frees this S buffer: the last wait
+            w = mbar_wait(bar_kfull + 8 * s, (g / C::NK) & 1u, s_abort, limit);
+            if (w == WAIT_OK && t >= 2) w = mbar_wait(bar_pvdone + 8 * b, ((g - 2u) >> 1) & 1u, s_abort, limit);
             if (w != WAIT_OK) break;
             tc_fence_after();
             const uint64_t kd = kdesc0 + ((s * C::QK_TILE_BYTES) >> 4);

@@ -196,9 +196,10 @@ class Protocol:
                 g = base + t
                 s = g % self.nk
                 b, use = self.buffer_of(g, t, bb)
+                # the kernel's order: the data-ready barrier first, the one that frees S[b] last
+                yield ("wait", f"kfull{s}", g // self.nk)
                 if t >= 2 and self.mut != "qk_skips_pvdone":
                     yield ("wait", f"pvdone{b}", use - 1)
-                yield ("wait", f"kfull{s}", g // self.nk)
                 if self.S_busy[b]:
                     raise AssertionError(f"hazard: QK({g}) writes S{b} while {sorted(self.S_busy[b])} run")
                 if self.S[b] is not None and self.S[b][0] == "P" and not self.S[b][2]:
@@ -227,8 +228,8 @@ class Protocol:
                 b, use = self.buffer_of(g, t, bb)
                 if self.alt and b != grp:
                     continue  # the other group's tile
+                yield ("wait", f"vfull{s}", g // self.nv)  # V lands first; P is the last wait
                 yield ("wait", f"pfull{b}{grp}", use)
-                yield ("wait", f"vfull{s}", g // self.nv)
                 if self.S[b] is None or self.S[b][:2] != ("P", g):
                     raise AssertionError(f"hazard: PV{grp}({g}) finds {self.S[b]} in S{b}")
                 if self.V[s] != g:
