@@ -223,8 +223,16 @@ __global__ void __launch_bounds__(kRouteThreads) sol_route_kernel(const __grid_c
   __syncthreads();
 
   // (2) proxy scores: warp w takes key blocks w, w + 8, ...; lane l holds components [l DPL, (l+1) DPL)
+  // of every q_bar in registers for the whole loop (re-reading them from shared memory for each key
+  // block would make shared-memory bandwidth the bound)
   {
     constexpr int DPL = D / 32;
+    float qv[R][DPL];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+#pragma unroll
+      for (int k = 0; k < DPL; ++k) qv[r][k] = r < nr ? s_qbar[r * D + lane * DPL + k] : 0.f;
+    }
     const float* kb = p.kbar + static_cast<size_t>(bh) * nkb * D + lane * DPL;
     constexpr int U = 4;  // key blocks in flight per warp
     for (int j0 = warp; j0 < nkb; j0 += kRouteWarps * U) {
@@ -253,11 +261,9 @@ __global__ void __launch_bounds__(kRouteThreads) sol_route_kernel(const __grid_c
           // the same fp32 operation order as the fused kernel's own routing, so both give the
           // same keep bits
           if constexpr (DPL == 4) {
-            const float4 qv = *reinterpret_cast<const float4*>(s_qbar + r * D + lane * DPL);
-            dot[r] = fmaf(qv.x, kv[u][0], fmaf(qv.y, kv[u][1], fmaf(qv.z, kv[u][2], qv.w * kv[u][3])));
+            dot[r] = fmaf(qv[r][0], kv[u][0], fmaf(qv[r][1], kv[u][1], fmaf(qv[r][2], kv[u][2], qv[r][3] * kv[u][3])));
           } else {
-            const float2 qv = *reinterpret_cast<const float2*>(s_qbar + r * D + lane * DPL);
-            dot[r] = fmaf(qv.x, kv[u][0], qv.y * kv[u][1]);
+            dot[r] = fmaf(qv[r][0], kv[u][0], qv[r][1] * kv[u][1]);
           }
         }
         butterfly_sum<R>(dot, lane);
