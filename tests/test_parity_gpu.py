@@ -260,11 +260,13 @@ def _header_only_workspace(B, H, device):
     return torch.zeros(((4 + B * H) * 4 + 255) // 256 * 256, dtype=torch.uint8, device=device)
 
 
-@pytest.mark.parametrize("L,d,H", [(3000, 128, 3), (1500, 64, 2), (262_221, 128, 1), (524_288, 64, 1)])
+@pytest.mark.parametrize("L,d,H", [(3000, 128, 3), (1500, 64, 2), (150_000, 128, 1), (140_000, 64, 1),
+                                   (262_221, 128, 1), (524_288, 64, 1)])
 def test_routing_pass_matches_in_kernel_routing(L, d, H):
     """Both routing paths do the same fp32 arithmetic in the same order, so the mask, the density
-    and O agree bit for bit. N_kb = 2049 and 4096 (the limit) run the routing pass with 4 query
-    blocks per CTA; sampled query blocks of those are also checked against the oracle."""
+    and O agree bit for bit. The routing pass takes 16 query blocks per CTA up to N_kb = 1024, 8 up
+    to 2048 (N_kb = 1172 and 1094 here) and 4 beyond (N_kb = 2049 and 4096, the limit); sampled
+    query blocks of the long cases are also checked against the oracle."""
     Qh, Kh, Vh = local_inputs(1, H, L, d, seed=L % 997 + d)
     Q, K, V = (torch.from_numpy(x).to(torch.bfloat16).cuda() for x in (Qh, Kh, Vh))
     kbar, vbar, klp, vlp = sa.sol_attn_pool(K, V, 128)
