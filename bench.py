@@ -386,7 +386,9 @@ def measure_config(name, dev, stream, pk, parity_units=4):
     torch.cuda.synchronize()
     kept = int(mask.to(torch.int64).sum())
     flops = kept_tile_flops(kept, w)
-    ms = timed(tau, 5)
+    # the clocks of this workload's own timed calls (long launches run longer under the power cap)
+    with ClockSampler(local_gpu_index(torch, dev.index if dev.index is not None else 0)) as clk:
+        ms = timed(tau, 5)
     spans = cta_spans(lambda: fwd(tau), dev, torch, sa)
     dense_ms = timed([math.inf] * H, 3)
     fwd(tau)  # leave the timed density's output in O for the parity sample
@@ -400,7 +402,8 @@ def measure_config(name, dev, stream, pk, parity_units=4):
     out = {"B": B, "H": H, "L": L, "d": d, "block": blk, "n_force": w.n_force, "density_target": key,
            "density": kept / float(B * H * nb * nb), "kept_tiles": kept, "fwd_ms": ms, "fwd_tflops": achieved,
            "frac": achieved / pk["bf16_tflops"], "dense_fwd_ms": dense_ms, "speedup_vs_dense": dense_ms / ms,
-           "cta_balance": spans, "parity_sample": sample_parity(collected, gpu_rows, mask_rows)}
+           "cta_balance": spans, "parity_sample": sample_parity(collected, gpu_rows, mask_rows),
+           "clocks": clk.summary()}
     del Q, K, V, O, ws, kbar, vbar, klp, vlp, mask
     torch.cuda.empty_cache()
     return out
