@@ -91,7 +91,6 @@ template <int D, bool QK8, bool PV8 = false>
 struct TcCfg {
   static constexpr int NCHUNK = D / 64;                 // 128-byte swizzle atoms per bf16 row
   static constexpr int CHUNK_BYTES = kRows * 128;       // 128 rows x 128 B
-  static constexpr int TILE_BYTES = NCHUNK * CHUNK_BYTES;
   static constexpr int QK_CHUNKS = QK8 ? D / 128 : NCHUNK;  // swizzle atoms per Q or K row
   static constexpr int QK_TILE_BYTES = QK_CHUNKS * CHUNK_BYTES;
   static constexpr int NK = (D == 128) ? 3 : 4;         // K ring depth
