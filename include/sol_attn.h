@@ -132,7 +132,9 @@ sol_status sol_attn_qknorm_rope_pool_qbar(const void* Q, const void* K, const vo
  * A code is the fp32 round-to-nearest-even of x * 127 / amax, clamped to [-127, 127]. Subtracting
  * mu shifts every logit of a query row by the same amount, so in exact arithmetic it changes
  * nothing; it keeps a common key offset out of the 8-bit range (SageAttention's smoothing).
- * d in {64, 128}, N_kb <= 4096, all pointers 16-byte aligned. Asynchronous on `stream`. */
+ * Errors, checked on the host before any launch: a non-positive size, a null or not 16-byte
+ * aligned pointer -> SOL_EINVAL; d not in {64, 128}, B*H > 65535 or N_kb > 4096 ->
+ * SOL_EUNSUPPORTED; a failed launch -> SOL_ECUDA. Asynchronous on `stream`. */
 sol_status sol_attn_quantize_qk8(const void* Q, const void* K, const float* kbar, int B, int H, int L,
                                  int d, int8_t* q8, int8_t* k8, int8_t* kbar8, float* q_scale,
                                  float* k_scale, float* kbar_scale, float* mu, void* stream);
@@ -146,8 +148,10 @@ sol_status sol_attn_quantize_qk8(const void* Q, const void* K, const float* kbar
  *             round to nearest even, saturating; transposed (tokens contiguous), 0 past L
  *   vbar8t    device, out, uint8 (E4M3 codes) [B, H, d, 128 * ceil(N_kb / 128)]: vbar with the same
  *             channel scales, transposed, 0 past N_kb
- * d = 128, N_kb <= 4096, B*H <= 65535, all pointers non-null and 16-byte aligned. Asynchronous on
- * `stream`; v_scale doubles as the per-channel maximum while the pass runs. */
+ * Errors, checked on the host before any launch: a non-positive size, a null or not 16-byte
+ * aligned pointer -> SOL_EINVAL; d != 128, B*H > 65535 or N_kb > 4096 -> SOL_EUNSUPPORTED; a
+ * failed launch -> SOL_ECUDA. Asynchronous on `stream`; v_scale doubles as the per-channel maximum
+ * while the pass runs. */
 sol_status sol_attn_quantize_v8(const void* V, const float* vbar, int B, int H, int L, int d,
                                 uint8_t* v8t, uint8_t* vbar8t, float* v_scale, void* stream);
 
